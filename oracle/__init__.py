@@ -1,0 +1,14 @@
+"""fp64 CPU oracle for the sparse MLA prefill attend block (test infrastructure).
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import this package. The CUDA library never does.
+"""
+from .oracle import (  # noqa: F401
+    attend_rows,
+    build,
+    bf16_to_double,
+    e4m3_to_double,
+    prefill_rows,
+    project_rows,
+    upproject_rows,
+)
