@@ -1,0 +1,157 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) sparse MLA prefill attend block.
+ *
+ * The block is the full-sequence (prefill) path of multi-head latent
+ * attention as given on the DeepSeek-V3.2-Exp "Sparse attention" page
+ * (model.py 574-589, 607-608) and the Kimi K2 "Output projection" page:
+ *
+ *   [k_nope_h | v_h][t] = W_kvb,h . kv_latent[t]              (wkv_b, view, split)
+ *   k_h[t]              = k_nope_h[t] ++ k_pe[t]                (rotary key shared by heads)
+ *   z[s,h,t]            = scale * <q[s,h], k_h[t]>              (scores)
+ *   keep(s,t)           = t in topk_idx[s,:] and t <= s          (index mask + causal mask)
+ *   attn[s,h]           = sum_t softmax_t(z | keep) v_h[t]      (softmax, value mix)
+ *   out[s]              = flatten_h(attn[s]) . W_o              (wo(x.flatten(2)), Delta = o W_O)
+ *
+ * Conventions (all calls):
+ *  - Every pointer argument except `workspace`'s host-side size is a DEVICE
+ *    pointer owned by the caller, 16-byte aligned, on the current device.
+ *    The library allocates no device memory; scratch lives in `workspace`.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronise. Host-side argument checks
+ *    return a status synchronously, before anything is launched.
+ *  - bf16 is IEEE binary16-bfloat (1-8-7); e4m3 is OCP FP8 E4M3FN.
+ *  - Fixed head geometry: d_nope = 128, d_rope = 64, d_v = 128,
+ *    d_latent = 512, d_model = 7168 (any other value: MLA_ERR_UNSUPPORTED).
+ *    Any H >= 1, B >= 0, 0 <= T <= MLA_MAX_T. B*T == 0 is a no-op that
+ *    returns MLA_OK right after the geometry check (NULL pointers allowed).
+ *  - Inputs are read-only; outputs must not alias inputs or the workspace.
+ *  - Kernels that wait on on-chip barriers give up after a bounded time and
+ *    record an error word on the device instead of hanging; read it with
+ *    mla_device_status().
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* mla_stream_t;
+
+#define MLA_MAX_T 65536
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_NULL = 1,         /* a required pointer is NULL */
+  MLA_ERR_SHAPE = 2,        /* a size is out of range (negative, T > MLA_MAX_T, topk < 1) */
+  MLA_ERR_UNSUPPORTED = 3,  /* head geometry other than 128/64/128/512/7168, or no sm_100 device */
+  MLA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than mla_workspace_bytes() */
+  MLA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+  MLA_ERR_ALIGN = 6,        /* a pointer is not 16-byte aligned */
+  MLA_ERR_DEVICE = 7        /* a kernel recorded a device-side error (see mla_device_status) */
+} mla_status;
+
+typedef enum {
+  MLA_W_BF16 = 0,          /* weights stored as bf16 */
+  MLA_W_E4M3_BLOCK128 = 1  /* e4m3 codes, one fp32 scale per 128 x 128 block (Kimi K2
+                              "Down projection" page: fmt e4m3, weight_block_size [128, 128]) */
+} mla_wdtype;
+
+typedef struct {
+  int B, T, H;
+  int d_nope, d_rope, d_v, d_latent, d_model;
+  int topk;          /* entries per row of topk_idx (ignored when topk_idx == NULL) */
+  mla_wdtype wdtype; /* storage of W_kvb and W_o */
+} mla_dims;
+
+/* Entry points, for mla_workspace_bytes(). */
+#define MLA_ENTRY_KV_UPPROJECT 0
+#define MLA_ENTRY_ATTEND 1
+#define MLA_ENTRY_OUT_PROJECT 2
+#define MLA_ENTRY_PREFILL 3
+
+/* Device workspace bytes that `entry` needs for these dims (has_topk = 1
+ * if a topk_idx will be passed). 0 when nothing is needed or the dims are
+ * invalid. The library never allocates; the caller passes this much. */
+size_t mla_workspace_bytes(const mla_dims* dims, int entry, int has_topk);
+
+/* Step A2 -- W_kvb up-projection (DeepSeek-V3.2-Exp "Sparse attention",
+ * `kv = self.wkv_b(kv)`; W_kvb shape from the MLA init, kv_b_proj
+ * [H*(128+128), 512] stored [out, in]).
+ *   kv_latent : bf16 [B*T, 512] (post-RMSNorm latent)
+ *   W_kvb     : bf16 or e4m3 [H*256, 512]; row h*256+i is k_nope_h[i] for
+ *               i < 128 and v_h[i-128] otherwise
+ *   W_kvb_scale: fp32 [2H, 4] (block scales) for e4m3, else ignored
+ *   kvh_out   : bf16 [B*T, H*256], same column order as W_kvb's rows
+ * Uses the tcgen05 tensor-core GEMM; fp32 accumulation, bf16 rounding. */
+int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_kvb,
+                     const float* W_kvb_scale, void* kvh_out, void* workspace,
+                     size_t ws_bytes, mla_stream_t stream);
+
+/* Steps A0-A5 -- up-projection, then sparse-causal attention
+ * (DeepSeek-V3.2-Exp "Sparse attention": scores, index mask + causal mask,
+ * softmax, value mix). Stops before W_o.
+ *   q        : bf16 [B, T, H, 192]: 128 non-rotary dims then 64 rotary dims
+ *   kv_latent: bf16 [B, T, 512]
+ *   k_pe     : bf16 [B, T, 64], rotated, shared by all heads
+ *   W_kvb, W_kvb_scale: as for mla_kv_upproject
+ *   topk_idx : int32 [B, T, topk] key indices per query, any order; NULL =
+ *              causal mask only (top-k >= T). Duplicates select once;
+ *              entries outside [0, T) select nothing; entries > s are
+ *              removed by the causal mask.
+ *   scale    : softmax scale applied to q.k (192^-0.5 for these models)
+ *   attn_out : bf16 [B, T, H, 128]. A query with no surviving key gets 0.
+ * Softmax in fp32 (exp2 form); P and V enter the PV product as bf16. */
+int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent,
+               const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
+               const int32_t* topk_idx, float scale, void* attn_out,
+               void* workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* Step A6 -- output projection (Kimi K2 / DeepSeek-V3.2-Exp "Output
+ * projection": Delta_attn = o W_O, no bias).
+ *   attn : bf16 [B*T, H*128] (heads flattened, h*128 + d)
+ *   W_o  : bf16 or e4m3 [H*128, 7168] (math orientation [in, out]; a
+ *          checkpoint's [out, in] weight is transposed once at load)
+ *   W_o_scale: fp32 [H, 56] block scales for e4m3, else ignored
+ *   out  : bf16 [B*T, 7168] */
+int mla_out_project(const mla_dims* dims, const void* attn, const void* W_o,
+                    const float* W_o_scale, void* out, void* workspace,
+                    size_t ws_bytes, mla_stream_t stream);
+
+/* The whole block: mla_attend followed by mla_out_project, with the
+ * attention output kept in the workspace. out: bf16 [B, T, 7168]. */
+int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent,
+                const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
+                const void* W_o, const float* W_o_scale, const int32_t* topk_idx,
+                float scale, void* out, void* workspace, size_t ws_bytes,
+                mla_stream_t stream);
+
+/* Human-readable text of a status code (static storage). */
+const char* mla_status_str(int status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device. *device_error receives 0 (none) or the code a kernel
+ * recorded (1xx: pipeline wait timed out; 2xx: bad launch geometry). Returns
+ * MLA_ERR_CUDA if synchronisation fails, else MLA_OK. */
+int mla_device_status(mla_stream_t stream, int* device_error);
+
+/* Per-kernel device timing (CUDA events on the launching stream).
+ * mla_profile_begin() starts recording events around every launch made by
+ * the calls above on this host thread's library instance; mla_profile_end()
+ * synchronises those events and writes, per kernel class, the total
+ * milliseconds and launch count, then stops recording.
+ * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention,
+ * 4 W_o GEMM. Arrays must hold MLA_PROFILE_CLASSES entries. */
+#define MLA_PROFILE_CLASSES 5
+int mla_profile_begin(void);
+int mla_profile_end(float* ms_total, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

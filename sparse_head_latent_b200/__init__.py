@@ -1,0 +1,28 @@
+"""B200 (sm_100a) sparse MLA prefill attend block.
+
+The C ABI (include/mla.h, libmla_b200.so) runs the whole block in CUDA
+kernels: W_kvb up-projection (tcgen05 GEMM), top-k selection bitmap,
+fused sparse-causal attention, W_o output projection (tcgen05 GEMM).
+This package is its thin ctypes binding; the library is loaded on first
+use and a missing build is an error, never a fallback.
+"""
+from .mla import (  # noqa: F401
+    MLA_ENTRY_ATTEND,
+    MLA_ENTRY_KV_UPPROJECT,
+    MLA_ENTRY_OUT_PROJECT,
+    MLA_ENTRY_PREFILL,
+    MlaDims,
+    MlaError,
+    library_path,
+    load_library,
+    make_dims,
+    mla_attend,
+    mla_device_status,
+    mla_kv_upproject,
+    mla_out_project,
+    mla_prefill,
+    mla_profile_begin,
+    mla_profile_end,
+    mla_status_str,
+    mla_workspace_bytes,
+)

@@ -1,0 +1,344 @@
+// attn.cuh -- fused sparse-causal MLA attention for sm_100a (tcgen05 + TMA).
+//
+// For one batch b, one head h and one tile of 128 queries s, over the key
+// blocks (128 keys each) in which some query of the tile selected a key
+// (DeepSeek-V3.2-Exp "Sparse attention", prefill):
+//   S   = q_h . [k_nope_h | k_pe]^T              (UMMA, K = 192, S in tensor memory)
+//   S   = -inf where bit(s, t) = 0                (top-k + causal selection)
+//   m,l = running max / sum of exp2(S*scale*log2e - m) per query row (fp32)
+//   O  += P . v_h                                 (UMMA, P bf16 in shared memory, O in tensor memory)
+//   attn[b, s, h, :] = O / l                      (bf16)
+// Neither the [T, T] scores nor a float mask is ever materialised: the
+// selection arrives as one bit per causal (query, key) pair.
+//
+// CTA = 192 threads:
+//   warp 0      TMA producer: Q once; K (k_nope from the up-projected kv
+//               plus the shared k_pe) into a 2-deep ring; V single-buffered
+//   warp 1      tensor-memory allocator and UMMA issuer; issues QK^T of the
+//               next block before PV of the current one so the tensor core
+//               works while the softmax runs
+//   warps 2..5  softmax: one query row per thread (tensor-memory lane)
+// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384).
+#pragma once
+
+#include "prepass.cuh"
+#include "ptx.cuh"
+
+namespace mla {
+
+struct AttnParams {
+  int B, T, H, nq;
+  float scale_log2;             // softmax scale * log2(e)
+  const uint4* bitmap;          // selection bitmap, NULL = causal mask only
+  const int32_t* blocks;        // active key blocks per tile (with bitmap)
+  __nv_bfloat16* attn;          // [B, T, H, 128]
+  int* err;
+};
+
+struct AttnSmem {
+  static constexpr int Q = 0;              // 3 x [128 x 64] bf16, 128B-swizzled
+  static constexpr int K0 = 49152;         // stage 0: k_nope 0-63, 64-127, k_pe
+  static constexpr int K1 = 98304;         // stage 1
+  static constexpr int V = 147456;         // 2 x [128 keys x 64 dv]
+  static constexpr int P = 180224;         // 2 x [128 rows x 64 keys]
+  static constexpr int BARS = 212992;
+  static constexpr int NUM_BARS = 13;
+  static constexpr int BYTES = 1024 + BARS + NUM_BARS * 8 + 16;
+};
+
+// Barrier slots.
+enum : int {
+  kBarQFull = 0, kBarKFull0 = 1, kBarKEmpty0 = 3, kBarVFull = 5, kBarSFull0 = 6,
+  kBarSFree0 = 8, kBarPFull = 10, kBarPvDone = 11, kBarDrain = 12
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(192, 1)
+sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+                       const __grid_constant__ CUtensorMap tmKpe, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::BARS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + AttnSmem::NUM_BARS);
+  int* abort_word = reinterpret_cast<int*>(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+
+  // Work item: heavy (late) query tiles first.
+  const int per_tile = p.B * p.H;
+  const int qt = p.nq - 1 - static_cast<int>(blockIdx.x) / per_tile;
+  const int rem = static_cast<int>(blockIdx.x) % per_tile;
+  const int b = rem / p.H, h = rem % p.H;
+  const int32_t* blist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.nq + qt) * (p.nq + 1) : nullptr;
+  const int n = blist ? blist[0] : qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQFull), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarKFull0 + i), 1);
+      mbar_init(bar(kBarKEmpty0 + i), 1);
+      mbar_init(bar(kBarSFull0 + i), 1);
+      mbar_init(bar(kBarSFree0 + i), 4);
+    }
+    mbar_init(bar(kBarVFull), 1);
+    mbar_init(bar(kBarPFull), 4);
+    mbar_init(bar(kBarPvDone), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_word = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmKV);
+    prefetch_tmap(&tmKpe);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_word, p.err};
+  const uint32_t sQ = smem_u32(smem + AttnSmem::Q);
+  const uint32_t sV = smem_u32(smem + AttnSmem::V);
+  const uint32_t sP = smem_u32(smem + AttnSmem::P);
+
+  if (warp == 0) {
+    if (lane == 0 && n > 0) {
+      // ---------------- TMA producer
+      int nk = 0, nv = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(bar(kBarQFull), 3 * 16384);
+      for (int c = 0; c < 3; ++c) tma_load_3d(sQ + c * 16384, &tmQ, bar(kBarQFull), h * 192 + 64 * c, qt * 128, b);
+      auto load_k = [&](int j) -> bool {
+        const int ks = j & 1;
+        if (!mbar_wait(bar(kBarKEmpty0 + ks), ((j >> 1) & 1) ^ 1, ab, kErrWaitMma)) return false;
+        const int t0 = (blist ? blist[1 + j] : j) * 128;
+        const uint32_t dst = smem_u32(smem + (ks ? AttnSmem::K1 : AttnSmem::K0));
+        const uint32_t fb = bar(kBarKFull0 + ks);
+        mbar_arrive_expect_tx(fb, 3 * 16384);
+        tma_load_3d(dst, &tmKV, fb, h * 256, t0, b);
+        tma_load_3d(dst + 16384, &tmKV, fb, h * 256 + 64, t0, b);
+        tma_load_3d(dst + 32768, &tmKpe, fb, 0, t0, b);
+        ++nk;
+        return true;
+      };
+      ok = load_k(0);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n && !(ok = load_k(j + 1))) break;
+        if (j >= 1 && !(ok = mbar_wait(bar(kBarPvDone), (j - 1) & 1, ab, kErrWaitMma))) break;
+        const int t0 = (blist ? blist[1 + j] : j) * 128;
+        mbar_arrive_expect_tx(bar(kBarVFull), 2 * 16384);
+        tma_load_3d(sV, &tmKV, bar(kBarVFull), h * 256 + 128, t0, b);
+        tma_load_3d(sV + 16384, &tmKV, bar(kBarVFull), h * 256 + 192, t0, b);
+        ++nv;
+      }
+      if (!ok) {
+        mbar_wait_drain(bar(kBarQFull), 0);
+        for (int i = (nk > 2 ? nk - 2 : 0); i < nk; ++i) mbar_wait_drain(bar(kBarKFull0 + (i & 1)), (i >> 1) & 1);
+        if (nv > 0) mbar_wait_drain(bar(kBarVFull), (nv - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n > 0) {
+      // ---------------- UMMA issuer
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+      bool ok = mbar_wait(bar(kBarQFull), 0, ab, kErrWaitTma);
+      int issued = 0;
+      auto issue_qk = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(bar(kBarKFull0 + st), (j >> 1) & 1, ab, kErrWaitTma)) return false;
+        if (!mbar_wait(bar(kBarSFree0 + st), ((j >> 1) & 1) ^ 1, ab, kErrWaitSoftmax)) return false;
+        tc_fence_after();
+        const uint32_t sK = smem_u32(smem + (st ? AttnSmem::K1 : AttnSmem::K0));
+        const uint32_t d = tmem + st * 128;
+#pragma unroll
+        for (int k = 0; k < 12; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idesc_qk,
+                  k > 0 ? 1u : 0u);
+        }
+        ++issued;
+        umma_commit(bar(kBarKEmpty0 + st));
+        umma_commit(bar(kBarSFull0 + st));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
+        if (!(ok = mbar_wait(bar(kBarPFull), j & 1, ab, kErrWaitSoftmax))) break;
+        if (!(ok = mbar_wait(bar(kBarVFull), j & 1, ab, kErrWaitTma))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t adesc = smem_desc_sw128(sP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(sV + k * 2048, 16384, 1024);
+          umma_ss(tmem + 256, adesc, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        ++issued;
+        umma_commit(bar(kBarPvDone));
+      }
+      if (!ok && issued > 0) {
+        umma_commit(bar(kBarDrain));
+        mbar_wait_drain(bar(kBarDrain), 0);
+      }
+    }
+  } else {
+    // ---------------- softmax warps: thread = query row r of the tile
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + static_cast<int>(lane);
+    const int s = qt * 128 + r;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int64_t tri_total = tri_index(p.nq, 0);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    uint8_t* prow0 = smem + AttnSmem::P + r * 128;
+    const uint32_t sw = lane & 7;  // 128B swizzle phase of this row
+
+    for (int j = 0; j < n; ++j) {
+      const int kb = blist ? blist[1 + j] : j;
+      uint32_t bw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (p.bitmap) {
+        const uint4 v = __ldg(p.bitmap + (static_cast<int64_t>(b) * tri_total + tri_index(qt, kb)) * 128 + r);
+        bw[0] = v.x; bw[1] = v.y; bw[2] = v.z; bw[3] = v.w;
+      }
+      const int st = j & 1;
+      if (!(ok = warp_wait(bar(kBarSFull0 + st), (j >> 1) & 1, ab, kErrWaitMma))) break;
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t a0[32], a1[32];
+        tmem_ld32x2(trow + st * 128, trow + st * 128 + 32, a0, a1);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(a0[c]); x[32 + c] = __uint_as_float(a1[c]); }
+        tmem_ld32x2(trow + st * 128 + 64, trow + st * 128 + 96, a0, a1);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) { x[64 + c] = __uint_as_float(a0[c]); x[96 + c] = __uint_as_float(a1[c]); }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarSFree0 + st));
+
+      // Scale into the log2 domain and apply the selection.
+      const bool all_sel = (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu;
+      const bool causal_diag = (p.bitmap == nullptr) && (kb == qt);
+      float mblk = -INFINITY;
+      if (__all_sync(0xffffffffu, all_sel && !causal_diag)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) { x[c] *= p.scale_log2; mblk = fmaxf(mblk, x[c]); }
+      } else if (causal_diag) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          x[c] = (c <= r) ? x[c] * p.scale_log2 : -INFINITY;
+          mblk = fmaxf(mblk, x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          x[c] = ((bw[c >> 5] >> (c & 31)) & 1u) ? x[c] * p.scale_log2 : -INFINITY;
+          mblk = fmaxf(mblk, x[c]);
+        }
+      }
+      // Lazy rescaling: keep the running max unless the block max exceeds it
+      // by more than 8 (a factor of 256), so O is rarely touched.
+      const float m_new = fmaxf(m_run, mblk);
+      const bool resc = (m_new - m_run) > 8.f;
+      float alpha = 1.f;
+      if (resc) {
+        alpha = ex2_approx(m_run - m_new);
+        m_run = m_new;
+      }
+      const float base = (m_run == -INFINITY) ? 0.f : m_run;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        x[c] = ex2_approx(x[c] - base);
+        rs += x[c];
+      }
+      l_run = l_run * alpha + rs;
+
+      // PV of the previous block must be complete before O is rescaled and
+      // before the P buffer is overwritten.
+      if (j >= 1) {
+        if (!(ok = warp_wait(bar(kBarPvDone), (j - 1) & 1, ab, kErrWaitMma))) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(trow + 256 + c0, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(trow + 256 + c0, o);
+          }
+        }
+      }
+      // P (bf16) into the 128B-swizzled K-major layout: row r, keys in two
+      // 64-wide chunks of 16 KB.
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        uint4 v;
+        v.x = pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]);
+        v.y = pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]);
+        v.z = pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]);
+        v.w = pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]);
+        *reinterpret_cast<uint4*>(prow0 + (ch >> 3) * 16384 + (((ch & 7) ^ sw) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarPFull));
+    }
+
+    if (ok) {
+      __nv_bfloat16* dst = p.attn + ((static_cast<int64_t>(b) * p.T + s) * p.H + h) * 128;
+      if (n > 0) {
+        ok = warp_wait(bar(kBarPvDone), (n - 1) & 1, ab, kErrWaitMma);
+        if (ok) {
+          tc_fence_after();
+          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 64) {
+            uint32_t a0[32], a1[32];
+            tmem_ld32x2(trow + 256 + c0, trow + 256 + c0 + 32, a0, a1);
+            if (s < p.T) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                d4[i] = make_uint4(pack_bf16x2(__uint_as_float(a0[8 * i + 0]) * inv, __uint_as_float(a0[8 * i + 1]) * inv),
+                                   pack_bf16x2(__uint_as_float(a0[8 * i + 2]) * inv, __uint_as_float(a0[8 * i + 3]) * inv),
+                                   pack_bf16x2(__uint_as_float(a0[8 * i + 4]) * inv, __uint_as_float(a0[8 * i + 5]) * inv),
+                                   pack_bf16x2(__uint_as_float(a0[8 * i + 6]) * inv, __uint_as_float(a0[8 * i + 7]) * inv));
+                d4[4 + i] = make_uint4(pack_bf16x2(__uint_as_float(a1[8 * i + 0]) * inv, __uint_as_float(a1[8 * i + 1]) * inv),
+                                       pack_bf16x2(__uint_as_float(a1[8 * i + 2]) * inv, __uint_as_float(a1[8 * i + 3]) * inv),
+                                       pack_bf16x2(__uint_as_float(a1[8 * i + 4]) * inv, __uint_as_float(a1[8 * i + 5]) * inv),
+                                       pack_bf16x2(__uint_as_float(a1[8 * i + 6]) * inv, __uint_as_float(a1[8 * i + 7]) * inv));
+              }
+            }
+          }
+        }
+      } else if (s < p.T) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+        for (int i = 0; i < 16; ++i) d4[i] = make_uint4(0, 0, 0, 0);  // no surviving key
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace mla

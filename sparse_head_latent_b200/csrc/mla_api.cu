@@ -1,0 +1,504 @@
+// mla_api.cu -- host side of the C ABI declared in include/mla.h:
+// argument validation, workspace carving, TMA tensor-map encoding, launch
+// sequencing on the caller's stream, device error word and per-kernel
+// event timing. All kernels live in the headers included below (one
+// translation unit, so no relocatable device code is needed).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "../../include/mla.h"
+#include "attn.cuh"
+#include "dequant.cuh"
+#include "gemm.cuh"
+#include "prepass.cuh"
+#include "ptx.cuh"
+
+// Device error word: kernels record the first error code here.
+__device__ int g_mla_device_error;
+
+namespace {
+
+using mla::GemmCfg;
+
+constexpr int kDn = 128, kDr = 64, kDv = 128, kL = 512, kD = 7168;
+using GemmKvb = GemmCfg<256, false>;  // latent x W_kvb^T  (B stored [N, K])
+using GemmWo = GemmCfg<256, true>;    // attn x W_o         (B stored [K, N])
+
+// ------------------------------------------------------------------ device state
+
+struct DeviceState {
+  bool ready = false;
+  int status = MLA_OK;
+  int sms = 0;
+  int* err = nullptr;  // address of g_mla_device_error on this device
+};
+
+std::mutex g_mutex;
+std::vector<DeviceState> g_devices;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// One-time set-up per device: device checks, kernel attributes, address of
+// the error word. Returns an mla_status.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (static_cast<int>(g_devices.size()) <= dev) g_devices.resize(dev + 1);
+  DeviceState& st = g_devices[dev];
+  if (!st.ready) {
+    st.ready = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      st.status = MLA_ERR_CUDA;
+    } else if (prop.major != 10) {
+      st.status = MLA_ERR_UNSUPPORTED;  // built for sm_100a only
+    } else {
+      st.sms = prop.multiProcessorCount;
+      bool ok = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err), g_mla_device_error) == cudaSuccess;
+      ok = ok && cudaMemset(st.err, 0, sizeof(int)) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc_kernel<GemmKvb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      GemmKvb::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc_kernel<GemmWo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      GemmWo::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      mla::AttnSmem::BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::topk_bitmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      200 * 1024) == cudaSuccess;
+      if (ok && g_encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        ok = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+             q == cudaDriverEntryPointSuccess && fn != nullptr;
+        if (ok) g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+      st.status = ok ? MLA_OK : MLA_ERR_CUDA;
+    }
+  }
+  *out = &st;
+  return st.status;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+// Row-major bf16/u8 matrix [outer, inner] with a row pitch; box
+// [box_outer, box_inner]; 128-byte swizzle; out-of-range rows read as zero.
+bool map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+            uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 tensor [B, T, inner] (row pitch inner*2 bytes), box [1, 128, 64].
+bool map_3d_bt(CUtensorMap* m, const void* base, uint64_t inner, uint64_t T, uint64_t B) {
+  const cuuint64_t dims[3] = {inner, T, B};
+  const cuuint64_t strides[2] = {inner * 2, inner * 2 * T};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ profiling
+
+struct ProfRecord {
+  int cls;
+  cudaEvent_t start, stop;
+};
+
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+thread_local Profiler t_prof;
+
+// Runs `launch` on `stream`, bracketed by events when profiling is on.
+template <class F>
+int timed_launch(int cls, cudaStream_t stream, F&& launch) {
+  ProfRecord r{cls, nullptr, nullptr};
+  if (t_prof.on) {
+    r.start = t_prof.get();
+    r.stop = t_prof.get();
+    cudaEventRecord(r.start, stream);
+  }
+  launch();
+  const cudaError_t e = cudaGetLastError();
+  if (t_prof.on) {
+    cudaEventRecord(r.stop, stream);
+    t_prof.recs.push_back(r);
+  }
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ validation and workspace
+
+namespace {
+
+constexpr size_t kNone = ~size_t(0);
+constexpr int64_t kMaxRows = int64_t(1) << 24;  // B*T limit (int32 tile coordinates with margin)
+
+struct WsLayout {
+  size_t kvh = kNone, attn = kNone, bitmap = kNone, blocks = kNone, wkvb = kNone, wo = kNone;
+  size_t total = 0;
+};
+
+int check_dims(const mla_dims* d) {
+  if (d == nullptr) return MLA_ERR_NULL;
+  if (d->d_nope != kDn || d->d_rope != kDr || d->d_v != kDv || d->d_latent != kL || d->d_model != kD)
+    return MLA_ERR_UNSUPPORTED;
+  if (d->wdtype != MLA_W_BF16 && d->wdtype != MLA_W_E4M3_BLOCK128) return MLA_ERR_UNSUPPORTED;
+  if (d->B < 0 || d->T < 0 || d->H < 1 || d->T > MLA_MAX_T) return MLA_ERR_SHAPE;
+  if (static_cast<int64_t>(d->B) * d->T > kMaxRows) return MLA_ERR_SHAPE;
+  return MLA_OK;
+}
+
+WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
+  WsLayout w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t rows = static_cast<size_t>(d.B) * d.T;
+  const size_t H = d.H;
+  const size_t nq = (static_cast<size_t>(d.T) + 127) / 128;
+  const bool fp8 = d.wdtype == MLA_W_E4M3_BLOCK128;
+  const bool attend = entry == MLA_ENTRY_ATTEND || entry == MLA_ENTRY_PREFILL;
+  if (attend) {
+    w.kvh = take(rows * H * (kDn + kDv) * 2);
+    if (entry == MLA_ENTRY_PREFILL) w.attn = take(rows * H * kDv * 2);
+    if (has_topk) {
+      w.bitmap = take(static_cast<size_t>(d.B) * (nq * (nq + 1) / 2) * 128 * 16);
+      w.blocks = take(static_cast<size_t>(d.B) * nq * (nq + 1) * 4);
+    }
+  }
+  if (fp8 && (attend || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
+  if (fp8 && (entry == MLA_ENTRY_PREFILL || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+  w.total = off;
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+// ------------------------------------------------------------------ stage launchers
+
+int launch_dequant(const DeviceState* ds, const void* codes, const float* scale, void* out, int rows, int cols,
+                   cudaStream_t st) {
+  const int64_t groups = static_cast<int64_t>(rows) * (cols / 16);
+  const int64_t want = (groups + 255) / 256;
+  const int grid = static_cast<int>(want < int64_t(ds->sms) * 8 ? want : int64_t(ds->sms) * 8);
+  return timed_launch(1, st, [&] {
+    mla::dequant_e4m3_block128_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(codes), scale,
+                                                            static_cast<__nv_bfloat16*>(out), rows, cols);
+  });
+}
+
+int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const void* wkvb, void* kvh,
+                    cudaStream_t st) {
+  const int N = H * (kDn + kDv), K = kL;
+  CUtensorMap ta, tb, tc;
+  if (!map_2d(&ta, lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 128) ||
+      !map_2d(&tb, wkvb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, GemmKvb::BN) ||
+      !map_2d(&tc, kvh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const int tiles = ((M + 127) / 128) * (N / GemmKvb::BN);
+  const int grid = tiles < ds->sms ? tiles : ds->sms;
+  return timed_launch(2, st, [&] {
+    mla::gemm_bf16_tc_kernel<GemmKvb><<<grid, GemmKvb::THREADS, GemmKvb::SMEM_BYTES, st>>>(ta, tb, tc, M, N, K,
+                                                                                         ds->err);
+  });
+}
+
+int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const void* wo, void* out,
+                   cudaStream_t st) {
+  const int N = kD, K = H * kDv;
+  CUtensorMap ta, tb, tc;
+  if (!map_2d(&ta, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, 128) ||
+      !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64) ||
+      !map_2d(&tc, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const int tiles = ((M + 127) / 128) * (N / GemmWo::BN);
+  const int grid = tiles < ds->sms ? tiles : ds->sms;
+  return timed_launch(4, st, [&] {
+    mla::gemm_bf16_tc_kernel<GemmWo><<<grid, GemmWo::THREADS, GemmWo::SMEM_BYTES, st>>>(ta, tb, tc, M, N, K,
+                                                                                      ds->err);
+  });
+}
+
+int launch_prepass(const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks, cudaStream_t st) {
+  const int nq = (d.T + 127) / 128;
+  const size_t smem = static_cast<size_t>(nq) * (1 + 4 * mla::kPrepassWarps) * 4;
+  dim3 grid(nq, d.B);
+  return timed_launch(0, st, [&] {
+    mla::topk_bitmap_kernel<<<grid, 32 * mla::kPrepassWarps, smem, st>>>(
+        topk, d.T, d.topk, nq, static_cast<uint4*>(bitmap), static_cast<int32_t*>(blocks));
+  });
+}
+
+int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, const void* kvh, const void* k_pe,
+                     const void* bitmap, const void* blocks, float scale, void* attn, cudaStream_t st) {
+  CUtensorMap tq, tkv, tpe;
+  if (!map_3d_bt(&tq, q, static_cast<uint64_t>(d.H) * (kDn + kDr), d.T, d.B) ||
+      !map_3d_bt(&tkv, kvh, static_cast<uint64_t>(d.H) * (kDn + kDv), d.T, d.B) ||
+      !map_3d_bt(&tpe, k_pe, kDr, d.T, d.B))
+    return MLA_ERR_CUDA;
+  mla::AttnParams p;
+  p.B = d.B;
+  p.T = d.T;
+  p.H = d.H;
+  p.nq = (d.T + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.bitmap = static_cast<const uint4*>(bitmap);
+  p.blocks = static_cast<const int32_t*>(blocks);
+  p.attn = static_cast<__nv_bfloat16*>(attn);
+  p.err = ds->err;
+  const int64_t grid = static_cast<int64_t>(d.B) * p.nq * d.H;
+  return timed_launch(3, st, [&] {
+    mla::sparse_mla_attn_kernel<<<static_cast<unsigned>(grid), 192, mla::AttnSmem::BYTES, st>>>(tq, tkv, tpe, p);
+  });
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ C ABI
+
+namespace {
+
+int begin_call(const mla_dims* dims, int entry, bool has_topk, void* ws, size_t ws_bytes, DeviceState** ds,
+               WsLayout* lay) {
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  *lay = ws_layout(*dims, entry, has_topk);
+  if (lay->total > 0 && (ws == nullptr || ws_bytes < lay->total)) return MLA_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned16(ws)) return MLA_ERR_ALIGN;
+  return device_state(ds);
+}
+
+// Up-projection into kvh; dequantises W_kvb into the workspace first when
+// it is stored as e4m3.
+int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* lat,
+                  const void* W_kvb, const float* W_kvb_scale, void* kvh, cudaStream_t st) {
+  const void* wk = W_kvb;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    void* dq = ws_at(ws, lay.wkvb);
+    int rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st);
+    if (rc != MLA_OK) return rc;
+    wk = dq;
+  }
+  return launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, st);
+}
+
+int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* q,
+               const void* lat, const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
+               const int32_t* topk_idx, float scale, void* attn, cudaStream_t st) {
+  void* kvh = ws_at(ws, lay.kvh);
+  int rc = run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, st);
+  if (rc != MLA_OK) return rc;
+  void* bitmap = nullptr;
+  void* blocks = nullptr;
+  if (topk_idx != nullptr) {
+    bitmap = ws_at(ws, lay.bitmap);
+    blocks = ws_at(ws, lay.blocks);
+    rc = launch_prepass(d, topk_idx, bitmap, blocks, st);
+    if (rc != MLA_OK) return rc;
+  }
+  return launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, st);
+}
+
+int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* attn,
+                    const void* W_o, const float* W_o_scale, void* out, cudaStream_t st) {
+  const void* wo = W_o;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    void* dq = ws_at(ws, lay.wo);
+    int rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st);
+    if (rc != MLA_OK) return rc;
+    wo = dq;
+  }
+  return launch_gemm_wo(ds, d.B * d.T, d.H, attn, wo, out, st);
+}
+
+bool fp8_scales_ok(const mla_dims* d, const float* s) { return d->wdtype != MLA_W_E4M3_BLOCK128 || s != nullptr; }
+
+}  // namespace
+
+extern "C" {
+
+size_t mla_workspace_bytes(const mla_dims* dims, int entry, int has_topk) {
+  if (check_dims(dims) != MLA_OK || entry < MLA_ENTRY_KV_UPPROJECT || entry > MLA_ENTRY_PREFILL) return 0;
+  return ws_layout(*dims, entry, has_topk != 0).total;
+}
+
+int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_kvb, const float* W_kvb_scale,
+                     void* kvh_out, void* workspace, size_t ws_bytes, mla_stream_t stream) {
+  DeviceState* ds = nullptr;
+  WsLayout lay;
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!kv_latent || !W_kvb || !kvh_out || !fp8_scales_ok(dims, W_kvb_scale)) return MLA_ERR_NULL;
+  if (!aligned16(kv_latent) || !aligned16(W_kvb) || !aligned16(kvh_out) || !aligned16(W_kvb_scale))
+    return MLA_ERR_ALIGN;
+  rc = begin_call(dims, MLA_ENTRY_KV_UPPROJECT, false, workspace, ws_bytes, &ds, &lay);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  return run_upproject(ds, *dims, lay, workspace, kv_latent, W_kvb, W_kvb_scale, kvh_out,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent, const void* k_pe, const void* W_kvb,
+               const float* W_kvb_scale, const int32_t* topk_idx, float scale, void* attn_out, void* workspace,
+               size_t ws_bytes, mla_stream_t stream) {
+  DeviceState* ds = nullptr;
+  WsLayout lay;
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!q || !kv_latent || !k_pe || !W_kvb || !attn_out || !fp8_scales_ok(dims, W_kvb_scale)) return MLA_ERR_NULL;
+  if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return MLA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(attn_out) ||
+      !aligned16(W_kvb_scale) || !aligned16(topk_idx))
+    return MLA_ERR_ALIGN;
+  rc = begin_call(dims, MLA_ENTRY_ATTEND, topk_idx != nullptr, workspace, ws_bytes, &ds, &lay);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  return run_attend(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, attn_out,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_out_project(const mla_dims* dims, const void* attn, const void* W_o, const float* W_o_scale, void* out,
+                    void* workspace, size_t ws_bytes, mla_stream_t stream) {
+  DeviceState* ds = nullptr;
+  WsLayout lay;
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!attn || !W_o || !out || !fp8_scales_ok(dims, W_o_scale)) return MLA_ERR_NULL;
+  if (!aligned16(attn) || !aligned16(W_o) || !aligned16(out) || !aligned16(W_o_scale)) return MLA_ERR_ALIGN;
+  rc = begin_call(dims, MLA_ENTRY_OUT_PROJECT, false, workspace, ws_bytes, &ds, &lay);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  return run_out_project(ds, *dims, lay, workspace, attn, W_o, W_o_scale, out,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent, const void* k_pe, const void* W_kvb,
+                const float* W_kvb_scale, const void* W_o, const float* W_o_scale, const int32_t* topk_idx,
+                float scale, void* out, void* workspace, size_t ws_bytes, mla_stream_t stream) {
+  DeviceState* ds = nullptr;
+  WsLayout lay;
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!q || !kv_latent || !k_pe || !W_kvb || !W_o || !out || !fp8_scales_ok(dims, W_kvb_scale) ||
+      !fp8_scales_ok(dims, W_o_scale))
+    return MLA_ERR_NULL;
+  if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return MLA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(W_o) ||
+      !aligned16(out) || !aligned16(W_kvb_scale) || !aligned16(W_o_scale) || !aligned16(topk_idx))
+    return MLA_ERR_ALIGN;
+  rc = begin_call(dims, MLA_ENTRY_PREFILL, topk_idx != nullptr, workspace, ws_bytes, &ds, &lay);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* attn = ws_at(workspace, lay.attn);
+  rc = run_attend(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, attn, st);
+  if (rc != MLA_OK) return rc;
+  return run_out_project(ds, *dims, lay, workspace, attn, W_o, W_o_scale, out, st);
+}
+
+const char* mla_status_str(int status) {
+  switch (status) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_NULL: return "a required pointer is NULL";
+    case MLA_ERR_SHAPE: return "a size is out of range";
+    case MLA_ERR_UNSUPPORTED: return "unsupported head geometry, weight type or device";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case MLA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case MLA_ERR_DEVICE: return "a kernel recorded a device-side error";
+    default: return "unknown status";
+  }
+}
+
+int mla_device_status(mla_stream_t stream, int* device_error) {
+  if (device_error == nullptr) return MLA_ERR_NULL;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != MLA_OK) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ds->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v != 0 && cudaMemset(ds->err, 0, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  *device_error = v;
+  return MLA_OK;
+}
+
+int mla_profile_begin(void) {
+  for (auto& r : t_prof.recs) {
+    t_prof.pool.push_back(r.start);
+    t_prof.pool.push_back(r.stop);
+  }
+  t_prof.recs.clear();
+  t_prof.on = true;
+  return MLA_OK;
+}
+
+int mla_profile_end(float* ms_total, int* launches) {
+  if (ms_total == nullptr || launches == nullptr) return MLA_ERR_NULL;
+  for (int i = 0; i < MLA_PROFILE_CLASSES; ++i) {
+    ms_total[i] = 0.f;
+    launches[i] = 0;
+  }
+  int rc = MLA_OK;
+  for (auto& r : t_prof.recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      rc = MLA_ERR_CUDA;
+      continue;
+    }
+    ms_total[r.cls] += ms;
+    launches[r.cls] += 1;
+  }
+  for (auto& r : t_prof.recs) {
+    t_prof.pool.push_back(r.start);
+    t_prof.pool.push_back(r.stop);
+  }
+  t_prof.recs.clear();
+  t_prof.on = false;
+  return rc;
+}
+
+}  // extern "C"

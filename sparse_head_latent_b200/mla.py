@@ -1,0 +1,211 @@
+"""Python binding of the C ABI in include/mla.h (argument marshalling only).
+
+Every function here forwards device pointers, sizes and the current CUDA
+stream of torch to ``libmla_b200.so``; all arithmetic happens in the CUDA
+kernels. There is no fallback: if the library or a CUDA device is missing,
+the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL = 0, 1, 2, 3
+MLA_W_BF16, MLA_W_E4M3_BLOCK128 = 0, 1
+MLA_PROFILE_CLASSES = 5
+PROFILE_CLASS_NAMES = ("topk_prepass", "weight_dequant", "gemm_kvb", "attention", "gemm_wo")
+D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL = 128, 64, 128, 512, 7168
+
+
+class MlaDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("d_nope", ctypes.c_int), ("d_rope", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("d_latent", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("topk", ctypes.c_int), ("wdtype", ctypes.c_int)]
+
+
+class MlaError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: status {status} ({mla_status_str(status)})")
+        self.status = status
+
+
+# Exported symbols with their C signatures (checked by the tests).
+_VP, _SZ = ctypes.c_void_p, ctypes.c_size_t
+SIGNATURES = {
+    "mla_workspace_bytes": (_SZ, [ctypes.POINTER(MlaDims), ctypes.c_int, ctypes.c_int]),
+    "mla_kv_upproject": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mla_attend": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_float,
+                                  _VP, _VP, _SZ, _VP]),
+    "mla_out_project": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "mla_prefill": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                   ctypes.c_float, _VP, _VP, _SZ, _VP]),
+    "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int)]),
+    "mla_profile_begin": (ctypes.c_int, []),
+    "mla_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
+}
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libmla_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"CUDA library not built: {_LIB_PATH} is missing "
+                                   "(run python -m sparse_head_latent_b200.build)")
+            lib = ctypes.CDLL(_LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(lib, name)
+                f.restype, f.argtypes = res, args
+            _lib = lib
+    return _lib
+
+
+def mla_status_str(status: int) -> str:
+    return load_library().mla_status_str(int(status)).decode()
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MlaError(fn, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(B, T, H, topk=0, fp8=False) -> MlaDims:
+    return MlaDims(int(B), int(T), int(H), D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL, int(topk),
+                   MLA_W_E4M3_BLOCK128 if fp8 else MLA_W_BF16)
+
+
+def _wtype(w: torch.Tensor) -> bool:
+    if w.dtype == torch.uint8:
+        return True
+    if w.dtype == torch.bfloat16:
+        return False
+    raise ValueError("weights must be bf16 or uint8 (e4m3 codes)")
+
+
+def mla_workspace_bytes(dims: MlaDims, entry: int, has_topk: bool) -> int:
+    return int(load_library().mla_workspace_bytes(ctypes.byref(dims), int(entry), 1 if has_topk else 0))
+
+
+def _workspace(dims, entry, has_topk, workspace, device):
+    need = mla_workspace_bytes(dims, entry, has_topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def mla_kv_upproject(kv_latent, W_kvb, W_kvb_scale=None, kvh_out=None, workspace=None, stream=None):
+    """kv_latent bf16 [..., 512] -> kvh bf16 [rows, H*256]."""
+    rows = kv_latent.numel() // D_LATENT
+    H = W_kvb.shape[0] // (D_NOPE + D_V)
+    dims = make_dims(1, rows, H, 0, _wtype(W_kvb))
+    if kvh_out is None:
+        kvh_out = torch.empty(rows, H * (D_NOPE + D_V), dtype=torch.bfloat16, device=kv_latent.device)
+    ws, nbytes = _workspace(dims, MLA_ENTRY_KV_UPPROJECT, False, workspace, kv_latent.device)
+    lib = load_library()
+    _check("mla_kv_upproject", lib.mla_kv_upproject(ctypes.byref(dims), _ptr(kv_latent), _ptr(W_kvb),
+                                                    _ptr(W_kvb_scale), _ptr(kvh_out), _ptr(ws), nbytes,
+                                                    _stream(stream)))
+    return kvh_out
+
+
+def mla_attend(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale=192 ** -0.5,
+               attn_out=None, workspace=None, stream=None):
+    """q [B,T,H,192], kv_latent [B,T,512], k_pe [B,T,64] (bf16) -> attn bf16 [B,T,H,128]."""
+    B, T, H, _ = q.shape
+    topk = 0 if topk_idx is None else topk_idx.shape[-1]
+    dims = make_dims(B, T, H, topk, _wtype(W_kvb))
+    if topk_idx is not None and topk_idx.dtype != torch.int32:
+        raise ValueError("topk_idx must be int32")
+    if attn_out is None:
+        attn_out = torch.empty(B, T, H, D_V, dtype=torch.bfloat16, device=q.device)
+    ws, nbytes = _workspace(dims, MLA_ENTRY_ATTEND, topk_idx is not None, workspace, q.device)
+    lib = load_library()
+    _check("mla_attend", lib.mla_attend(ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb),
+                                        _ptr(W_kvb_scale), _ptr(topk_idx), float(scale), _ptr(attn_out),
+                                        _ptr(ws), nbytes, _stream(stream)))
+    return attn_out
+
+
+def mla_out_project(attn, W_o, W_o_scale=None, out=None, workspace=None, stream=None):
+    """attn bf16 [rows, H*128] (or [B,T,H,128]) -> out bf16 [rows, 7168]."""
+    H = W_o.shape[0] // D_V
+    rows = attn.numel() // (H * D_V)
+    dims = make_dims(1, rows, H, 0, _wtype(W_o))
+    if out is None:
+        out = torch.empty(rows, D_MODEL, dtype=torch.bfloat16, device=attn.device)
+    ws, nbytes = _workspace(dims, MLA_ENTRY_OUT_PROJECT, False, workspace, attn.device)
+    lib = load_library()
+    _check("mla_out_project", lib.mla_out_project(ctypes.byref(dims), _ptr(attn), _ptr(W_o), _ptr(W_o_scale),
+                                                  _ptr(out), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk_idx=None,
+                scale=192 ** -0.5, out=None, workspace=None, stream=None):
+    """The whole attend block: -> out bf16 [B, T, 7168]."""
+    B, T, H, _ = q.shape
+    topk = 0 if topk_idx is None else topk_idx.shape[-1]
+    fp8 = _wtype(W_kvb)
+    if _wtype(W_o) != fp8:
+        raise ValueError("W_kvb and W_o must use the same storage type")
+    if topk_idx is not None and topk_idx.dtype != torch.int32:
+        raise ValueError("topk_idx must be int32")
+    dims = make_dims(B, T, H, topk, fp8)
+    if out is None:
+        out = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=q.device)
+    ws, nbytes = _workspace(dims, MLA_ENTRY_PREFILL, topk_idx is not None, workspace, q.device)
+    lib = load_library()
+    _check("mla_prefill", lib.mla_prefill(ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb),
+                                          _ptr(W_kvb_scale), _ptr(W_o), _ptr(W_o_scale), _ptr(topk_idx),
+                                          float(scale), _ptr(out), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def mla_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word."""
+    v = ctypes.c_int(0)
+    _check("mla_device_status", load_library().mla_device_status(_stream(stream), ctypes.byref(v)))
+    return v.value
+
+
+def mla_profile_begin():
+    _check("mla_profile_begin", load_library().mla_profile_begin())
+
+
+def mla_profile_end():
+    """{class name: (total ms, launches)} for the launches since mla_profile_begin()."""
+    ms = (ctypes.c_float * MLA_PROFILE_CLASSES)()
+    n = (ctypes.c_int * MLA_PROFILE_CLASSES)()
+    _check("mla_profile_end", load_library().mla_profile_end(ms, n))
+    return {PROFILE_CLASS_NAMES[i]: (float(ms[i]), int(n[i])) for i in range(MLA_PROFILE_CLASSES)}

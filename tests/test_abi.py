@@ -1,0 +1,122 @@
+"""The C ABI library loads, exports what include/mla.h declares, and rejects
+bad arguments on the host before touching a device (CPU only)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_head_latent_b200 as mla
+from sparse_head_latent_b200 import build as cuda_build
+from sparse_head_latent_b200.mla import SIGNATURES, MlaDims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    cuda_build.build()
+    return mla.load_library()
+
+
+def test_header_declares_the_bound_entry_points():
+    assert _declared() == sorted(SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", mla.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mla_[a-z_0-9]+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def _dims(**kw):
+    d = mla.make_dims(1, 256, 4, 16, False)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_workspace_sizes(lib):
+    d = _dims()
+    kvh = 256 * 4 * 256 * 2
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_KV_UPPROJECT, False) == 0
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_OUT_PROJECT, False) == 0
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, False) == kvh
+    with_topk = mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, True)
+    nq = 2
+    bitmap = nq * (nq + 1) // 2 * 128 * 16
+    assert with_topk == kvh + bitmap + 256 * ((nq * (nq + 1) * 4 + 255) // 256)
+    pre = mla.mla_workspace_bytes(d, mla.MLA_ENTRY_PREFILL, True)
+    assert pre == with_topk + 256 * 4 * 128 * 2
+    d8 = _dims(wdtype=1)
+    assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_KV_UPPROJECT, False) == 4 * 256 * 512 * 2
+    assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_OUT_PROJECT, False) == 4 * 128 * 7168 * 2
+    assert mla.mla_workspace_bytes(_dims(d_model=4096), mla.MLA_ENTRY_ATTEND, False) == 0
+    assert mla.mla_workspace_bytes(d, 9, False) == 0
+
+
+def _attend(lib, d, ptrs=None, scale=0.07, ws=None, nbytes=0):
+    p = dict(q=16, lat=16, kpe=16, wk=16, sc=None, tk=None, out=16)
+    p.update(ptrs or {})
+    return lib.mla_attend(ctypes.byref(d), p["q"], p["lat"], p["kpe"], p["wk"], p["sc"], p["tk"],
+                          ctypes.c_float(scale), p["out"], ws, nbytes, None)
+
+
+def test_host_validation_before_any_device_work(lib):
+    # Every case below is rejected by host checks that run before the first
+    # CUDA call, so they run without a GPU.
+    assert _attend(lib, _dims(d_nope=64)) == 3                 # unsupported geometry
+    assert _attend(lib, _dims(wdtype=5)) == 3
+    assert _attend(lib, _dims(T=-1)) == 2                      # bad size
+    assert _attend(lib, _dims(T=70000)) == 2                   # above MLA_MAX_T
+    assert _attend(lib, _dims(H=0)) == 2
+    assert _attend(lib, _dims(), {"q": None}) == 1             # NULL input
+    assert _attend(lib, _dims(wdtype=1)) == 1                  # e4m3 without scales
+    assert _attend(lib, _dims(topk=0), {"tk": 16}) == 2        # top-k rows of width 0
+    assert _attend(lib, _dims(), scale=float("nan")) == 2
+    assert _attend(lib, _dims(), {"q": 24}) == 6               # misaligned
+    assert _attend(lib, _dims()) == 4                          # workspace missing
+    assert _attend(lib, _dims(), ws=16, nbytes=100) == 4       # workspace too small
+    d = _dims()
+    assert lib.mla_prefill(ctypes.byref(d), 16, 16, 16, 16, None, None, None, None, ctypes.c_float(0.1),
+                           16, None, 0, None) == 1              # W_o NULL
+    assert lib.mla_out_project(None, 16, 16, None, 16, None, 0, None) == 1
+    assert lib.mla_kv_upproject(ctypes.byref(_dims(d_latent=256)), 16, 16, None, 16, None, 0, None) == 3
+    # An empty problem is a no-op, even with NULL pointers and no workspace.
+    assert _attend(lib, _dims(T=0), {"q": None, "out": None}) == 0
+    assert lib.mla_prefill(ctypes.byref(_dims(B=0)), None, None, None, None, None, None, None, None,
+                           ctypes.c_float(0.1), None, None, 0, None) == 0
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert mla.mla_status_str(code)
+    assert mla.mla_status_str(0) == "ok"
+    assert "unknown" in mla.mla_status_str(99)
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 4, 1, 192, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mla.mla_attend(q, torch.zeros(1, 4, 512, dtype=torch.bfloat16), torch.zeros(1, 4, 64, dtype=torch.bfloat16),
+                       torch.zeros(256, 512, dtype=torch.bfloat16), workspace=torch.zeros(1, dtype=torch.uint8))
+
+
+def test_dims_struct_matches_header():
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct \{(.*?)\} mla_dims;", src, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\b([A-Za-z_]+)\s*[,;]", body)
+    assert names == [f for f, _ in MlaDims._fields_]

@@ -1,0 +1,192 @@
+"""CUDA path vs the fp64 oracle, element by element (needs a B200).
+
+Every call goes through the C ABI (libmla_b200.so) via the ctypes binding.
+Tolerances: max-abs <= 2e-2 and relative L2 <= 5e-3 on the attention output
+and on the projected output (and on the up-projected kv, which feeds both).
+Small cases are compared in full; they span several 128-row tiles and a
+ragged tail.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+mla = pytest.importorskip("sparse_head_latent_b200")
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 2e-2, 5e-3
+
+
+def _dev(x):
+    return {k: v.cuda() for k, v in x.tensors().items()}
+
+
+def assert_close(got, ref, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    d = got - ref
+    max_abs = float(np.abs(d).max()) if d.size else 0.0
+    nref = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(d) / nref) if nref > 0 else float(np.linalg.norm(d))
+    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
+    return max_abs, rel
+
+
+def _no_device_error():
+    assert mla.mla_device_status() == 0
+
+
+def _attend(x, g, topk_idx="inputs"):
+    tk = g.get("topk_idx") if isinstance(topk_idx, str) else topk_idx
+    return mla.mla_attend(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g.get("W_kvb_scale"),
+                          topk_idx=tk, scale=x.scale)
+
+
+# ---------------------------------------------------------------- GEMM stages
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("B,T,H", [(1, 128, 1), (2, 300, 4), (1, 1000, 2)])
+def test_upprojection_matches_oracle(B, T, H, fp8):
+    x = synth.make_inputs(0, B=B, T=T, H=H, topk=None, seed=21, fp8=fp8)
+    g = _dev(x)
+    kvh = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"], g.get("W_kvb_scale"))
+    _no_device_error()
+    ref = oracle.upproject_rows(x, range(B * T))
+    assert_close(kvh.float().cpu().numpy(), ref, "kvh")
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("rows,H", [(128, 1), (300, 4), (517, 2)])
+def test_output_projection_matches_oracle(rows, H, fp8):
+    x = synth.make_inputs(0, T=8, H=H, topk=None, seed=22, fp8=fp8)
+    gen = torch.Generator().manual_seed(rows)
+    attn = (0.05 * torch.randn(rows, H * 128, generator=gen)).to(torch.bfloat16)
+    g = _dev(x)
+    out = mla.mla_out_project(attn.cuda(), g["W_o"], g.get("W_o_scale"))
+    _no_device_error()
+    ref = oracle.project_rows(x, attn.to(torch.float64).numpy())
+    assert_close(out.float().cpu().numpy(), ref, "out")
+
+
+# ---------------------------------------------------------------- attention
+
+ATTEND_CASES = {
+    "tiny_sparse": dict(B=1, T=128, H=8, topk=32),
+    "ragged_sparse": dict(B=2, T=300, H=3, topk=40),
+    "ragged_causal": dict(B=1, T=300, H=2, topk=None),
+    "short_rows": dict(B=1, T=77, H=2, topk=100),
+    "four_tiles": dict(B=1, T=512, H=2, topk=96),
+    "fp8_sparse": dict(B=2, T=200, H=2, topk=24, fp8=True),
+}
+
+
+@pytest.mark.parametrize("case", sorted(ATTEND_CASES))
+def test_attend_matches_oracle(case):
+    c = dict(ATTEND_CASES[case])
+    x = synth.make_inputs(0, seed=31, **c)
+    g = _dev(x)
+    attn = _attend(x, g)
+    _no_device_error()
+    ref = oracle.attend_rows(x, range(x.B * x.T))
+    assert_close(attn.float().cpu().numpy().reshape(ref.shape), ref, case)
+
+
+def test_topk_listing_every_key_equals_causal_only():
+    x = synth.make_inputs(0, B=1, T=260, H=2, topk=260, seed=32)
+    g = _dev(x)
+    full = _attend(x, g)
+    causal = _attend(x, g, topk_idx=None)
+    _no_device_error()
+    assert torch.equal(full, causal)
+    ref = oracle.attend_rows(x, range(x.T))
+    assert_close(causal.float().cpu().numpy().reshape(ref.shape), ref, "causal")
+
+
+def test_order_duplicates_and_out_of_range_entries():
+    x = synth.make_inputs(0, B=2, T=256, H=2, topk=20, seed=33)
+    g = _dev(x)
+    base = _attend(x, g)
+    tk = x.topk_idx.clone()
+    gen = torch.Generator().manual_seed(3)
+    perm = torch.rand(tk.shape, generator=gen).argsort(-1)
+    shuffled = tk.gather(-1, perm)
+    doubled = torch.cat([shuffled, shuffled.flip(-1)], dim=-1).contiguous()
+    assert torch.equal(base, _attend(x, g, topk_idx=doubled.cuda()))
+    # Entries above s never survive; out-of-range values in their place change nothing.
+    s_idx = torch.arange(x.T)[None, :, None]
+    bad = torch.tensor([-1, -9, x.T, 1 << 30], dtype=torch.int32)
+    fill = bad[torch.arange(tk.numel()).reshape(tk.shape) % 4]
+    tk_bad = torch.where(tk > s_idx, fill, tk).contiguous()
+    assert torch.equal(base, _attend(x, g, topk_idx=tk_bad.cuda()))
+    _no_device_error()
+    x.topk_idx = tk_bad
+    ref = oracle.attend_rows(x, range(x.B * x.T))
+    assert_close(base.float().cpu().numpy().reshape(ref.shape), ref, "dups/out-of-range")
+
+
+def test_rows_without_any_key_are_zero():
+    x = synth.make_inputs(0, B=1, T=384, H=2, topk=8, seed=34)
+    tk = x.topk_idx.clone()
+    tk[0, 130:260] = -1                      # a whole tile and parts of two more
+    x.topk_idx = tk
+    g = _dev(x)
+    attn = _attend(x, g)
+    _no_device_error()
+    assert not attn[0, 130:260].any()
+    ref = oracle.attend_rows(x, range(x.T))
+    assert_close(attn.float().cpu().numpy().reshape(ref.shape), ref, "empty rows")
+
+
+def test_single_selected_key_returns_its_value():
+    x = synth.make_inputs(0, B=1, T=200, H=2, topk=4, seed=35)
+    x.topk_idx = torch.full_like(x.topk_idx, 150)
+    g = _dev(x)
+    attn = _attend(x, g)
+    kvh = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"]).view(x.T, 2, 256)
+    _no_device_error()
+    assert not attn[0, :150].any()
+    # softmax over one key is exactly 1, so attn equals the stored bf16 v (up to
+    # the final bf16 rounding of a value that is already bf16).
+    v = kvh[150, :, 128:]
+    assert torch.equal(attn[0, 150:], v.unsqueeze(0).expand(50, 2, 128))
+
+
+# ---------------------------------------------------------------- whole block
+
+@pytest.mark.parametrize("case", ["tiny_sparse", "ragged_sparse", "ragged_causal", "fp8_sparse"])
+def test_prefill_matches_oracle(case):
+    c = dict(ATTEND_CASES[case])
+    x = synth.make_inputs(0, seed=41, **c)
+    g = _dev(x)
+    out = mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g.get("W_kvb_scale"),
+                          g.get("W_o_scale"), topk_idx=g.get("topk_idx"), scale=x.scale)
+    _no_device_error()
+    rows = list(range(x.B * x.T))
+    ref_attn, ref_out = oracle.prefill_rows(x, rows)
+    assert_close(out.float().cpu().numpy().reshape(len(rows), 7168), ref_out, case)
+
+
+def test_prefill_equals_attend_then_out_project():
+    x = synth.make_inputs(0, B=1, T=256, H=4, topk=32, seed=42)
+    g = _dev(x)
+    out = mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], topk_idx=g["topk_idx"],
+                          scale=x.scale)
+    attn = _attend(x, g)
+    out2 = mla.mla_out_project(attn, g["W_o"])
+    _no_device_error()
+    assert torch.equal(out.view(-1, 7168), out2)
+
+
+def test_empty_problem_is_a_noop():
+    x = synth.make_inputs(0, B=1, T=4, H=2, topk=2, seed=43)
+    g = _dev(x)
+    q0 = g["q"][:, :0].contiguous()
+    attn = mla.mla_attend(q0, g["kv_latent"][:, :0].contiguous(), g["k_pe"][:, :0].contiguous(), g["W_kvb"],
+                          topk_idx=g["topk_idx"][:, :0].contiguous(), scale=x.scale)
+    assert attn.shape == (1, 0, 2, 128)
+    _no_device_error()
