@@ -1,0 +1,443 @@
+"""Benchmark of the sparse MLA prefill attend block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+
+One step = one mla_prefill call (W_kvb up-projection, top-k bitmap,
+sparse-causal attention, W_o) over one batch of seeded synthetic inputs of
+the chosen workload (default: DeepSeek-V3.2-Exp-shaped sparse prefill,
+B=1, T=4096, H=128, top-k 2048). With N > 1 (torchrun, one rank per GPU)
+every rank runs its own independent instance: the work shards by sequence
+with no collective on the data path ("weak" scaling); the time is the max
+over ranks.
+
+Metric: algorithmic TFLOP/s (the method's own work: up-projection, the
+selected causal (query, key) pairs only, output projection), plus
+queries/s and the fraction of the measured bf16 tensor peak. Rank 0 prints
+one JSON line. ``--impl reference`` times the fp64 CPU oracle on the host
+cores instead (the reference arm; a deliberately slow program).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "sparse MLA prefill TFLOP/s and queries/s (T=4096,H=128,top-k 2048); % of bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("ptx.cuh", "gemm.cuh", "attn.cuh", "prepass.cuh", "dequant.cuh", "mla_api.cu")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--config", type=int, default=1)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer run (default: --steps)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------------ work model
+
+def selected_pairs(x) -> int:
+    """Sum over queries of |A_s| = |{t in topk_idx[b,s,:] : 0 <= t <= s}| (distinct)."""
+    if x.topk_idx is None:
+        return x.B * x.T * (x.T + 1) // 2
+    total = 0
+    s = torch.arange(x.T, dtype=torch.int64)[:, None]
+    for b in range(x.B):
+        for lo in range(0, x.T, 512):
+            tk = x.topk_idx[b, lo:lo + 512].to(torch.int64)
+            ok = (tk >= 0) & (tk <= s[lo:lo + 512])
+            v = torch.where(ok, tk, torch.full_like(tk, -1)).sort(dim=1).values
+            distinct = (v[:, 1:] != v[:, :-1]) & (v[:, 1:] >= 0)
+            total += int(distinct.sum()) + int((v[:, 0] >= 0).sum())
+    return total
+
+
+def work_model(x):
+    M, H = x.B * x.T, x.H
+    pairs = selected_pairs(x)
+    f_kvb = 2.0 * M * 512 * H * 256
+    f_attn = float(pairs) * H * (2 * 192 + 2 * 128)
+    f_wo = 2.0 * M * H * 128 * 7168
+    wbytes = 1 if x.fp8 else 2
+    comp = (x.q.numel() * 2 + x.kv_latent.numel() * 2 + x.k_pe.numel() * 2
+            + x.W_kvb.numel() * wbytes + x.W_o.numel() * wbytes
+            + (x.W_kvb_scale.numel() * 4 + x.W_o_scale.numel() * 4 if x.fp8 else 0)
+            + (x.topk_idx.numel() * 4 if x.topk_idx is not None else 0) + M * 7168 * 2)
+    return dict(pairs=pairs, flops_kvb=f_kvb, flops_attn=f_attn, flops_wo=f_wo,
+                flops=f_kvb + f_attn + f_wo, compulsory_bytes=comp)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_head_latent_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                    and parts[3] == src:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu, self.period = gpu_index, period_ms
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 f"-lms={self.period}", f"--id={self.gpu}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle sampling
+
+def oracle_unit(x, rng):
+    """One sampled unit of the workload for the CPU oracle: a random
+    (query row, head) pair, its attention over the selected keys (with the
+    up-projection of those keys for that head) and that head's share of the
+    output projection. Returns (seconds, algorithmic flops of the unit)."""
+    import oracle
+    b = int(rng.integers(0, x.B))
+    s = int(rng.integers(0, x.T))
+    h = int(rng.integers(0, x.H))
+    row = b * x.T + s
+    if x.topk_idx is None:
+        n_sel = s + 1
+    else:
+        tk = x.topk_idx[b, s]
+        n_sel = int(torch.unique(tk[(tk >= 0) & (tk <= s)]).numel())
+    t0 = time.perf_counter()
+    a = oracle.attend_rows(x, [row], heads=[h])
+    full = np.zeros((1, x.H * 128))
+    full[0, h * 128:(h + 1) * 128] = a[0, 0]
+    oracle.project_rows(x, full)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * 512 * 256 + n_sel * (2 * 192 + 2 * 128) + 2.0 * 128 * 7168
+    return dt, flops
+
+
+def cpu_baseline(x, budget_s: float, seed: int = 7):
+    rng = np.random.default_rng(seed)
+    tot_t, tot_f, n = 0.0, 0.0, 0
+    while tot_t < budget_s and n < 10000:
+        dt, fl = oracle_unit(x, rng)
+        tot_t += dt
+        tot_f += fl
+        n += 1
+    return {"value": tot_f / tot_t / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} random (query row, head) units of {x.name}: fp64 up-projection of the row's "
+                      f"selected keys for that head, masked softmax, value mix and the head's slice of W_o; "
+                      f"{tot_t:.1f} s on 1 host thread",
+            "seconds": tot_t}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (a no-op on one rank)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local):
+    import sparse_head_latent_b200 as mla
+
+    cfg = synth.CONFIGS[args.config]
+    x = synth.make_inputs(args.config)
+    wm = work_model(x)
+    dev = torch.device("cuda", local)
+    g = {k: v.to(dev) for k, v in x.tensors().items()}
+    dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8)
+    ws_bytes = mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_PREFILL, x.topk_idx is not None)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(x.B, x.T, 7168, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g.get("W_kvb_scale"),
+                        g.get("W_o_scale"), topk_idx=g.get("topk_idx"), scale=x.scale, out=out,
+                        workspace=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if mla.mla_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    clocks = ClockSampler(local).start()
+    time.sleep(0.3)
+    # ---- device-resident timing (with per-kernel events)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mla.mla_profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = mla.mla_profile_end()
+    t_wall1 = time.time()
+    barrier(world)
+    ms_local = e0.elapsed_time(e1) / args.steps
+    if mla.mla_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or args.steps
+    host_in = {k: g[k].cpu().pin_memory() for k in ("q", "kv_latent", "k_pe", "topk_idx") if g.get(k) is not None}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            g[k].copy_(t, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall2 = time.time()
+    barrier(world)
+    e2e_ms_local = f0.elapsed_time(f1) / e2e_steps
+    time.sleep(0.2)
+    clocks.stop()
+
+    ms = max_over_ranks(ms_local, world)
+    e2e_ms = max_over_ranks(e2e_ms_local, world)
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    tflops = wm["flops"] * world / (ms * 1e-3) / 1e12
+    qps = x.B * x.T * world / (ms * 1e-3)
+    e2e_tflops = wm["flops"] * world / (e2e_ms * 1e-3) / 1e12
+    # Per-kernel algorithmic work per launch.
+    kflops = {"gemm_kvb": wm["flops_kvb"], "attention": wm["flops_attn"], "gemm_wo": wm["flops_wo"]}
+    per_kernel = {}
+    for name, (tot_ms, n) in prof.items():
+        if n == 0:
+            continue
+        avg = tot_ms / n
+        d = {"launches": n, "avg_ms": round(avg, 5)}
+        if name in kflops:
+            d["tflops"] = round(kflops[name] / (avg * 1e-3) / 1e12, 1)
+        per_kernel[name] = d
+    dom = max((k for k in per_kernel if k in kflops), key=lambda k: prof[k][0])
+    dom_avg_ms = prof[dom][0] / prof[dom][1]
+    achieved = kflops[dom] / (dom_avg_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roof_t = max(wm["flops"] / (peak * 1e12), wm["compulsory_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    clk = clocks.summary(t_wall0, t_wall2)
+    result = {
+        "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the workload; no checkpoint)",
+        "config": {"workload": cfg["name"], "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
+                   "weights": "e4m3 block-128" if x.fp8 else "bf16", "parallelism": f"independent sequences x{world}",
+                   "l2": "no flush: every step reads > 600 MB, inputs larger than the 126 MB L2"},
+        "queries_per_s": round(qps, 1),
+        "frac_of_bf16_peak": round(tflops / world / peak, 4),
+        "frac_of_roofline": round(roof_t / (ms * 1e-3), 4),
+        "algorithmic_gflop_per_step": round(wm["flops"] / 1e9, 2),
+        "selected_pairs": wm["pairs"],
+        "per_kernel": per_kernel,
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(dom, cfg["name"]),
+                     "peak_source": f"{peak_src} bf16 dense (burst), MEASURED_PEAKS.json"},
+        "e2e": {"value": round(e2e_tflops, 2), "unit": UNIT, "h2d_bytes_per_step": h2d * world,
+                "d2h_bytes_per_step": d2h * world, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": int(sum(n for _, n in prof.values())),
+        "clocks": clk,
+        "pages_note": "the source pages give only shapes and parameter counts: no throughput numbers or hardware",
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = {k: v for k, v in cpu_baseline(x, args.cpu_seconds).items() if k != "seconds"}
+    return result
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    x = synth.make_inputs(args.config)
+    rng = np.random.default_rng(11)
+    # Each step is one sampled (query row, head) unit; about 0.2 s each at
+    # this workload, so a default run stays within a few minutes.
+    for _ in range(args.warmup):
+        oracle_unit(x, rng)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_unit(x, rng)
+        tot_t += dt
+        tot_f += fl
+    v = tot_f / tot_t / 1e12
+    sample = f"{args.steps} random (query row, head) units of {cfg['name']} (fp64 oracle, 1 host thread)"
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": cfg["name"], "B": x.B, "T": x.T, "H": x.H,
+                                                    "topk": x.topk},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+    else:
+        rank, world, local = dist_setup()
+        try:
+            res = run_ours(args, rank, world, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

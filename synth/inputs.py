@@ -108,8 +108,15 @@ def quantize_e4m3_block128(w: torch.Tensor, g: torch.Generator):
 
 
 def make_topk(B: int, T: int, k: int, seed: int, rows_per_chunk: int = 256) -> torch.Tensor:
-    """topk_idx int32 [B, T, k] by the selection rule in the module docstring."""
-    assert 1 <= k <= T
+    """topk_idx int32 [B, T, k] by the selection rule in the module docstring.
+
+    With k > T the rows hold every key of [0, T) and then the k - T
+    positions T, T+1, ... (out of range, so they select nothing)."""
+    assert k >= 1
+    if k > T:
+        base = make_topk(B, T, T, seed, rows_per_chunk)
+        extra = torch.arange(T, k, dtype=torch.int32).expand(B, T, k - T)
+        return torch.cat([base, extra], dim=-1).contiguous()
     g = _gen(seed, _TID_TOPK)
     out = torch.empty(B, T, k, dtype=torch.int32)
     t = torch.arange(T, dtype=torch.int64)

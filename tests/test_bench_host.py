@@ -1,0 +1,93 @@
+"""Host-side logic of bench.py (CPU only): the work model, the max-over-ranks
+reduction on two gloo ranks, and the reference (CPU oracle) arm."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_selected_pairs_follow_the_topk_rule():
+    x = synth.make_inputs(0)
+    # min(k, s+1) distinct keys in [0, s] per row (the padding sits above s).
+    assert bench.selected_pairs(x) == sum(min(32, s + 1) for s in range(128))
+    x.topk_idx = torch.cat([x.topk_idx, x.topk_idx, torch.full_like(x.topk_idx, -3)], dim=-1)
+    assert bench.selected_pairs(x) == sum(min(32, s + 1) for s in range(128))
+    x.topk_idx = None
+    assert bench.selected_pairs(x) == 128 * 129 // 2
+
+
+def test_work_model_of_the_headline_workload():
+    x = synth.make_inputs(0, T=4096, H=1, topk=2048)  # H=1 keeps it cheap; FLOPs scale with H
+    wm = bench.work_model(x)
+    assert wm["pairs"] == 6_292_480
+    assert wm["flops_kvb"] == 2 * 4096 * 512 * 256
+    assert wm["flops_wo"] == 2 * 4096 * 128 * 7168
+    # At H=128 the three steps are 137.4 / 515.5 / 962.1 GFLOP.
+    assert abs(wm["flops_kvb"] * 128 / 1e9 - 137.4) < 0.1
+    assert abs(wm["flops_attn"] * 128 / 1e9 - 515.5) < 0.1
+    assert abs(wm["flops_wo"] * 128 / 1e9 - 962.1) < 0.1
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        q.put((rank, bench.max_over_ranks(1.5 + rank, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    got = dict(q.get(timeout=5) for _ in range(2))
+    assert got == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_prints_one_line_on_rank_zero_only():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "0", "--steps", "3",
+                        "--warmup", "1"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
+    env["RANK"], env["WORLD_SIZE"] = "1", "2"
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "0", "--steps", "3"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_cpu_baseline_sample_is_bounded():
+    x = synth.make_inputs(0)
+    d = bench.cpu_baseline(x, 0.5)
+    assert d["kind"] == "oracle" and d["cores"] == 1 and d["value"] > 0
+    assert d["seconds"] < 5
