@@ -53,7 +53,21 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer run (default: --steps)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    p.add_argument("--B", type=int, default=None, help="override the workload's batch (profiling runs)")
+    p.add_argument("--T", type=int, default=None, help="override the workload's sequence length")
+    p.add_argument("--H", type=int, default=None, help="override the workload's head count")
+    p.add_argument("--topk", type=int, default=None, help="override the workload's top-k")
     return p.parse_args(argv)
+
+
+def workload(args):
+    """(name, inputs) of the chosen config with any size overrides applied."""
+    cfg = dict(synth.CONFIGS[args.config])
+    over = {k: getattr(args, k) for k in ("B", "T", "H", "topk") if getattr(args, k) is not None}
+    name = cfg["name"]
+    if over:
+        name += "_" + "_".join(f"{k}{v}" for k, v in over.items())
+    return name, synth.make_inputs(args.config, **over)
 
 
 # ------------------------------------------------------------------ work model
@@ -268,8 +282,7 @@ def max_over_ranks(value: float, world: int) -> float:
 def run_ours(args, rank, world, local):
     import sparse_head_latent_b200 as mla
 
-    cfg = synth.CONFIGS[args.config]
-    x = synth.make_inputs(args.config)
+    name, x = workload(args)
     wm = work_model(x)
     dev = torch.device("cuda", local)
     g = {k: v.to(dev) for k, v in x.tensors().items()}
@@ -351,14 +364,14 @@ def run_ours(args, rank, world, local):
     # Per-kernel algorithmic work per launch.
     kflops = {"gemm_kvb": wm["flops_kvb"], "attention": wm["flops_attn"], "gemm_wo": wm["flops_wo"]}
     per_kernel = {}
-    for name, (tot_ms, n) in prof.items():
+    for kname, (tot_ms, n) in prof.items():
         if n == 0:
             continue
         avg = tot_ms / n
         d = {"launches": n, "avg_ms": round(avg, 5)}
-        if name in kflops:
-            d["tflops"] = round(kflops[name] / (avg * 1e-3) / 1e12, 1)
-        per_kernel[name] = d
+        if kname in kflops:
+            d["tflops"] = round(kflops[kname] / (avg * 1e-3) / 1e12, 1)
+        per_kernel[kname] = d
     dom = max((k for k in per_kernel if k in kflops), key=lambda k: prof[k][0])
     dom_avg_ms = prof[dom][0] / prof[dom][1]
     achieved = kflops[dom] / (dom_avg_ms * 1e-3) / 1e12
@@ -370,7 +383,7 @@ def run_ours(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the workload; no checkpoint)",
-        "config": {"workload": cfg["name"], "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
+        "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
                    "weights": "e4m3 block-128" if x.fp8 else "bf16", "parallelism": f"independent sequences x{world}",
                    "l2": "no flush: every step reads > 600 MB, inputs larger than the 126 MB L2"},
         "queries_per_s": round(qps, 1),
@@ -381,7 +394,7 @@ def run_ours(args, rank, world, local):
         "per_kernel": per_kernel,
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic(dom, cfg["name"]),
+                     "traffic": ncu_traffic(dom, name),
                      "peak_source": f"{peak_src} bf16 dense (burst), MEASURED_PEAKS.json"},
         "e2e": {"value": round(e2e_tflops, 2), "unit": UNIT, "h2d_bytes_per_step": h2d * world,
                 "d2h_bytes_per_step": d2h * world, "ms_per_step": round(e2e_ms, 4)},
@@ -399,8 +412,7 @@ def run_ours(args, rank, world, local):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    cfg = synth.CONFIGS[args.config]
-    x = synth.make_inputs(args.config)
+    name, x = workload(args)
     rng = np.random.default_rng(11)
     # Each step is one sampled (query row, head) unit; about 0.2 s each at
     # this workload, so a default run stays within a few minutes.
@@ -412,11 +424,11 @@ def run_reference(args, rank, world):
         tot_t += dt
         tot_f += fl
     v = tot_f / tot_t / 1e12
-    sample = f"{args.steps} random (query row, head) units of {cfg['name']} (fp64 oracle, 1 host thread)"
+    sample = f"{args.steps} random (query row, head) units of {name} (fp64 oracle, 1 host thread)"
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded)", "config": {"workload": cfg["name"], "B": x.B, "T": x.T, "H": x.H,
+            "data": "synthetic (seeded)", "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H,
                                                     "topk": x.topk},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -103,7 +103,8 @@ int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_
  *              causal mask only (top-k >= T). Duplicates select once;
  *              entries outside [0, T) select nothing; entries > s are
  *              removed by the causal mask.
- *   scale    : softmax scale applied to q.k (192^-0.5 for these models)
+ *   scale    : softmax scale applied to q.k, finite and > 0 (192^-0.5 for
+ *              these models)
  *   attn_out : bf16 [B, T, H, 128]. A query with no surviving key gets 0.
  * Softmax in fp32 (exp2 form); P and V enter the PV product as bf16. */
 int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent,

@@ -6,19 +6,21 @@
 //   S   = q_h . [k_nope_h | k_pe]^T              (UMMA, K = 192, S in tensor memory)
 //   S   = -inf where bit(s, t) = 0                (top-k + causal selection)
 //   m,l = running max / sum of exp2(S*scale*log2e - m) per query row (fp32)
-//   O  += P . v_h                                 (UMMA, P bf16 in shared memory, O in tensor memory)
+//   O  += P . v_h                                 (UMMA, P bf16 in tensor memory, O in tensor memory)
 //   attn[b, s, h, :] = O / l                      (bf16)
 // Neither the [T, T] scores nor a float mask is ever materialised: the
 // selection arrives as one bit per causal (query, key) pair.
 //
 // CTA = 192 threads:
 //   warp 0      TMA producer: Q once; K (k_nope from the up-projected kv
-//               plus the shared k_pe) into a 2-deep ring; V single-buffered
+//               plus the shared k_pe) and V into 2-deep rings
 //   warp 1      tensor-memory allocator and UMMA issuer; issues QK^T of the
 //               next block before PV of the current one so the tensor core
 //               works while the softmax runs
 //   warps 2..5  softmax: one query row per thread (tensor-memory lane)
-// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384).
+// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384), P [384,448)
+// (P: 128 bf16 per row packed in 64 columns; the PV UMMA reads it as its A
+// operand, so P never touches shared memory).
 #pragma once
 
 #include "prepass.cuh"
@@ -28,6 +30,7 @@ namespace mla {
 
 struct AttnParams {
   int B, T, H, nq;
+  int hgroup;                   // heads per scheduling group (divides H)
   float scale_log2;             // softmax scale * log2(e)
   const uint4* bitmap;          // selection bitmap, NULL = causal mask only
   const int32_t* blocks;        // active key blocks per tile (with bitmap)
@@ -39,17 +42,20 @@ struct AttnSmem {
   static constexpr int Q = 0;              // 3 x [128 x 64] bf16, 128B-swizzled
   static constexpr int K0 = 49152;         // stage 0: k_nope 0-63, 64-127, k_pe
   static constexpr int K1 = 98304;         // stage 1
-  static constexpr int V = 147456;         // 2 x [128 keys x 64 dv]
-  static constexpr int P = 180224;         // 2 x [128 rows x 64 keys]
+  static constexpr int V0 = 147456;        // stage 0: 2 x [128 keys x 64 dv]
+  static constexpr int V1 = 180224;        // stage 1
   static constexpr int BARS = 212992;
-  static constexpr int NUM_BARS = 13;
+  static constexpr int NUM_BARS = 16;
   static constexpr int BYTES = 1024 + BARS + NUM_BARS * 8 + 16;
 };
 
+// Tensor-memory columns.
+constexpr uint32_t kTmemS0 = 0, kTmemO = 256, kTmemP = 384;
+
 // Barrier slots.
 enum : int {
-  kBarQFull = 0, kBarKFull0 = 1, kBarKEmpty0 = 3, kBarVFull = 5, kBarSFull0 = 6,
-  kBarSFree0 = 8, kBarPFull = 10, kBarPvDone = 11, kBarDrain = 12
+  kBarQFull = 0, kBarKFull0 = 1, kBarKEmpty0 = 3, kBarVFull0 = 5, kBarVEmpty0 = 7, kBarSFull0 = 9,
+  kBarSFree0 = 11, kBarPFull = 13, kBarPvDone = 14, kBarDrain = 15
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -72,11 +78,15 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
 
-  // Work item: heavy (late) query tiles first.
-  const int per_tile = p.B * p.H;
-  const int qt = p.nq - 1 - static_cast<int>(blockIdx.x) / per_tile;
-  const int rem = static_cast<int>(blockIdx.x) % per_tile;
-  const int b = rem / p.H, h = rem % p.H;
+  // Work item. CTAs are ordered by groups of `hgroup` heads, so that the
+  // CTAs resident at any time read the K/V of a few heads and those stay in
+  // L2; within a group, heavy (late) query tiles come first.
+  const int per_group = p.nq * p.B * p.hgroup;
+  const int hg = static_cast<int>(blockIdx.x) / per_group;
+  const int rem0 = static_cast<int>(blockIdx.x) % per_group;
+  const int qt = p.nq - 1 - rem0 / (p.B * p.hgroup);
+  const int rem = rem0 % (p.B * p.hgroup);
+  const int b = rem / p.hgroup, h = hg * p.hgroup + rem % p.hgroup;
   const int32_t* blist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.nq + qt) * (p.nq + 1) : nullptr;
   const int n = blist ? blist[0] : qt + 1;
 
@@ -85,10 +95,11 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarKFull0 + i), 1);
       mbar_init(bar(kBarKEmpty0 + i), 1);
+      mbar_init(bar(kBarVFull0 + i), 1);
+      mbar_init(bar(kBarVEmpty0 + i), 1);
       mbar_init(bar(kBarSFull0 + i), 1);
       mbar_init(bar(kBarSFree0 + i), 4);
     }
-    mbar_init(bar(kBarVFull), 1);
     mbar_init(bar(kBarPFull), 4);
     mbar_init(bar(kBarPvDone), 1);
     mbar_init(bar(kBarDrain), 1);
@@ -110,8 +121,6 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_word, p.err};
   const uint32_t sQ = smem_u32(smem + AttnSmem::Q);
-  const uint32_t sV = smem_u32(smem + AttnSmem::V);
-  const uint32_t sP = smem_u32(smem + AttnSmem::P);
 
   if (warp == 0) {
     if (lane == 0 && n > 0) {
@@ -136,17 +145,20 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ok = load_k(0);
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n && !(ok = load_k(j + 1))) break;
-        if (j >= 1 && !(ok = mbar_wait(bar(kBarPvDone), (j - 1) & 1, ab, kErrWaitMma))) break;
+        const int vs = j & 1;
+        if (!(ok = mbar_wait(bar(kBarVEmpty0 + vs), ((j >> 1) & 1) ^ 1, ab, kErrWaitMma))) break;
         const int t0 = (blist ? blist[1 + j] : j) * 128;
-        mbar_arrive_expect_tx(bar(kBarVFull), 2 * 16384);
-        tma_load_3d(sV, &tmKV, bar(kBarVFull), h * 256 + 128, t0, b);
-        tma_load_3d(sV + 16384, &tmKV, bar(kBarVFull), h * 256 + 192, t0, b);
+        const uint32_t dst = smem_u32(smem + (vs ? AttnSmem::V1 : AttnSmem::V0));
+        const uint32_t fb = bar(kBarVFull0 + vs);
+        mbar_arrive_expect_tx(fb, 2 * 16384);
+        tma_load_3d(dst, &tmKV, fb, h * 256 + 128, t0, b);
+        tma_load_3d(dst + 16384, &tmKV, fb, h * 256 + 192, t0, b);
         ++nv;
       }
       if (!ok) {
         mbar_wait_drain(bar(kBarQFull), 0);
         for (int i = (nk > 2 ? nk - 2 : 0); i < nk; ++i) mbar_wait_drain(bar(kBarKFull0 + (i & 1)), (i >> 1) & 1);
-        if (nv > 0) mbar_wait_drain(bar(kBarVFull), (nv - 1) & 1);
+        for (int i = (nv > 2 ? nv - 2 : 0); i < nv; ++i) mbar_wait_drain(bar(kBarVFull0 + (i & 1)), (i >> 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -162,7 +174,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (!mbar_wait(bar(kBarSFree0 + st), ((j >> 1) & 1) ^ 1, ab, kErrWaitSoftmax)) return false;
         tc_fence_after();
         const uint32_t sK = smem_u32(smem + (st ? AttnSmem::K1 : AttnSmem::K0));
-        const uint32_t d = tmem + st * 128;
+        const uint32_t d = tmem + kTmemS0 + st * 128;
 #pragma unroll
         for (int k = 0; k < 12; ++k) {
           const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
@@ -177,16 +189,18 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       if (ok) ok = issue_qk(0);
       for (int j = 0; j < n && ok; ++j) {
         if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
+        const int vs = j & 1;
         if (!(ok = mbar_wait(bar(kBarPFull), j & 1, ab, kErrWaitSoftmax))) break;
-        if (!(ok = mbar_wait(bar(kBarVFull), j & 1, ab, kErrWaitTma))) break;
+        if (!(ok = mbar_wait(bar(kBarVFull0 + vs), (j >> 1) & 1, ab, kErrWaitTma))) break;
         tc_fence_after();
+        const uint32_t sV = smem_u32(smem + (vs ? AttnSmem::V1 : AttnSmem::V0));
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint64_t adesc = smem_desc_sw128(sP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(sV + k * 2048, 16384, 1024);
-          umma_ss(tmem + 256, adesc, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+          umma_ts(tmem + kTmemO, tmem + kTmemP + k * 8, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
         }
         ++issued;
+        umma_commit(bar(kBarVEmpty0 + vs));
         umma_commit(bar(kBarPvDone));
       }
       if (!ok && issued > 0) {
@@ -201,10 +215,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const int s = qt * 128 + r;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int64_t tri_total = tri_index(p.nq, 0);
-    float m_run = -INFINITY, l_run = 0.f;
+    const float c = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 domain) and sum
     bool ok = true;
-    uint8_t* prow0 = smem + AttnSmem::P + r * 128;
-    const uint32_t sw = lane & 7;  // 128B swizzle phase of this row
 
     for (int j = 0; j < n; ++j) {
       const int kb = blist ? blist[1 + j] : j;
@@ -219,37 +232,36 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       float x[128];
       {
         uint32_t a0[32], a1[32];
-        tmem_ld32x2(trow + st * 128, trow + st * 128 + 32, a0, a1);
+        tmem_ld32x2(trow + kTmemS0 + st * 128, trow + kTmemS0 + st * 128 + 32, a0, a1);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) { x[c] = __uint_as_float(a0[c]); x[32 + c] = __uint_as_float(a1[c]); }
-        tmem_ld32x2(trow + st * 128 + 64, trow + st * 128 + 96, a0, a1);
+        for (int i = 0; i < 32; ++i) { x[i] = __uint_as_float(a0[i]); x[32 + i] = __uint_as_float(a1[i]); }
+        tmem_ld32x2(trow + kTmemS0 + st * 128 + 64, trow + kTmemS0 + st * 128 + 96, a0, a1);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) { x[64 + c] = __uint_as_float(a0[c]); x[96 + c] = __uint_as_float(a1[c]); }
+        for (int i = 0; i < 32; ++i) { x[64 + i] = __uint_as_float(a0[i]); x[96 + i] = __uint_as_float(a1[i]); }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarSFree0 + st));
 
-      // Scale into the log2 domain and apply the selection.
+      // Selection: unselected scores become -inf (raw domain; the scale is
+      // positive, so the max commutes with it).
       const bool all_sel = (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu;
       const bool causal_diag = (p.bitmap == nullptr) && (kb == qt);
-      float mblk = -INFINITY;
-      if (__all_sync(0xffffffffu, all_sel && !causal_diag)) {
+      if (causal_diag) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) { x[c] *= p.scale_log2; mblk = fmaxf(mblk, x[c]); }
-      } else if (causal_diag) {
+        for (int i = 0; i < 128; ++i) x[i] = (i <= r) ? x[i] : -INFINITY;
+      } else if (!__all_sync(0xffffffffu, all_sel)) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          x[c] = (c <= r) ? x[c] * p.scale_log2 : -INFINITY;
-          mblk = fmaxf(mblk, x[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          x[c] = ((bw[c >> 5] >> (c & 31)) & 1u) ? x[c] * p.scale_log2 : -INFINITY;
-          mblk = fmaxf(mblk, x[c]);
-        }
+        for (int i = 0; i < 128; ++i) x[i] = ((bw[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
       }
+      // Row max with 8 independent chains.
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], x[i]);
+      const float mblk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
       // Lazy rescaling: keep the running max unless the block max exceeds it
       // by more than 8 (a factor of 256), so O is rarely touched.
       const float m_new = fmaxf(m_run, mblk);
@@ -260,16 +272,18 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         m_run = m_new;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
+      float sm[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2_approx(x[c] - base);
-        rs += x[c];
+      for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        x[i] = ex2_approx(fmaf(x[i], c, -base));
+        sm[i & 7] += x[i];
       }
-      l_run = l_run * alpha + rs;
+      l_run = l_run * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
 
       // PV of the previous block must be complete before O is rescaled and
-      // before the P buffer is overwritten.
+      // before P is overwritten.
       if (j >= 1) {
         if (!(ok = warp_wait(bar(kBarPvDone), (j - 1) & 1, ab, kErrWaitMma))) break;
         tc_fence_after();
@@ -277,25 +291,23 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll 1
           for (int c0 = 0; c0 < 128; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(trow + 256 + c0, o);
+            tmem_ld32(trow + kTmemO + c0, o);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(trow + 256 + c0, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(trow + kTmemO + c0, o);
           }
         }
       }
-      // P (bf16) into the 128B-swizzled K-major layout: row r, keys in two
-      // 64-wide chunks of 16 KB.
+      // P (bf16 pairs) into tensor memory, row r = lane r.
+      {
+        uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint4 v;
-        v.x = pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]);
-        v.y = pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]);
-        v.z = pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]);
-        v.w = pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]);
-        *reinterpret_cast<uint4*>(prow0 + (ch >> 3) * 16384 + (((ch & 7) ^ sw) << 4)) = v;
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        tmem_st32(trow + kTmemP, pk);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[64 + 2 * i], x[64 + 2 * i + 1]);
+        tmem_st32(trow + kTmemP + 32, pk);
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull));
@@ -311,7 +323,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll 1
           for (int c0 = 0; c0 < 128; c0 += 64) {
             uint32_t a0[32], a1[32];
-            tmem_ld32x2(trow + 256 + c0, trow + 256 + c0 + 32, a0, a1);
+            tmem_ld32x2(trow + kTmemO + c0, trow + kTmemO + c0 + 32, a0, a1);
             if (s < p.T) {
               uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll

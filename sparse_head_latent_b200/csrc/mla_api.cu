@@ -72,8 +72,8 @@ int device_state(DeviceState** out) {
                                       GemmWo::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AttnSmem::BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::topk_bitmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      200 * 1024) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::topk_bitmap_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      mla::kPrepassWarps * (MLA_MAX_T / 128) * 16) == cudaSuccess;
       if (ok && g_encode == nullptr) {
         cudaDriverEntryPointQueryResult q;
         void* fn = nullptr;
@@ -256,13 +256,22 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
   });
 }
 
-int launch_prepass(const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks, cudaStream_t st) {
+int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks,
+                   cudaStream_t st) {
+  (void)ds;
   const int nq = (d.T + 127) / 128;
-  const size_t smem = static_cast<size_t>(nq) * (1 + 4 * mla::kPrepassWarps) * 4;
+  const int64_t rows = static_cast<int64_t>(d.B) * nq * 128;
+  const unsigned grid_rows = static_cast<unsigned>((rows + mla::kPrepassWarps - 1) / mla::kPrepassWarps);
+  const size_t smem = static_cast<size_t>(mla::kPrepassWarps) * nq * 4 * 4;
+  int rc = timed_launch(0, st, [&] {
+    mla::topk_bitmap_rows_kernel<<<grid_rows, 32 * mla::kPrepassWarps, smem, st>>>(
+        topk, d.B, d.T, d.topk, nq, static_cast<uint4*>(bitmap));
+  });
+  if (rc != MLA_OK) return rc;
   dim3 grid(nq, d.B);
   return timed_launch(0, st, [&] {
-    mla::topk_bitmap_kernel<<<grid, 32 * mla::kPrepassWarps, smem, st>>>(
-        topk, d.T, d.topk, nq, static_cast<uint4*>(bitmap), static_cast<int32_t*>(blocks));
+    mla::topk_block_list_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4*>(bitmap), nq,
+                                                      static_cast<int32_t*>(blocks));
   });
 }
 
@@ -278,6 +287,15 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.T = d.T;
   p.H = d.H;
   p.nq = (d.T + 127) / 128;
+  // Heads per scheduling group: the largest of 8, 4, 2, 1 that divides H and
+  // keeps the group's K/V (T x 512 bytes per head and batch) near 48 MB or less.
+  p.hgroup = 1;
+  for (int g = 8; g > 1; g /= 2) {
+    if (d.H % g == 0 && static_cast<int64_t>(g) * d.B * d.T * 512 <= (int64_t(48) << 20)) {
+      p.hgroup = g;
+      break;
+    }
+  }
   p.scale_log2 = scale * 1.4426950408889634f;
   p.bitmap = static_cast<const uint4*>(bitmap);
   p.blocks = static_cast<const int32_t*>(blocks);
@@ -330,7 +348,7 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   if (topk_idx != nullptr) {
     bitmap = ws_at(ws, lay.bitmap);
     blocks = ws_at(ws, lay.blocks);
-    rc = launch_prepass(d, topk_idx, bitmap, blocks, st);
+    rc = launch_prepass(ds, d, topk_idx, bitmap, blocks, st);
     if (rc != MLA_OK) return rc;
   }
   return launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, st);
@@ -386,7 +404,7 @@ int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent, const
   if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
   if (!q || !kv_latent || !k_pe || !W_kvb || !attn_out || !fp8_scales_ok(dims, W_kvb_scale)) return MLA_ERR_NULL;
   if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
-  if (!std::isfinite(scale)) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MLA_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(attn_out) ||
       !aligned16(W_kvb_scale) || !aligned16(topk_idx))
     return MLA_ERR_ALIGN;
@@ -425,7 +443,7 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent, cons
       !fp8_scales_ok(dims, W_o_scale))
     return MLA_ERR_NULL;
   if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
-  if (!std::isfinite(scale)) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MLA_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(W_o) ||
       !aligned16(out) || !aligned16(W_kvb_scale) || !aligned16(W_o_scale) || !aligned16(topk_idx))
     return MLA_ERR_ALIGN;

@@ -11,10 +11,18 @@
 //   bitmap[b][qt*(qt+1)/2 + kb][row 0..127][4 x u32]   (bit c of the 128 = key kb*128 + c)
 //   blocks[b][qt][0] = number of key blocks with any bit set for the tile,
 //   blocks[b][qt][1 + i] = their indices, ascending.
-// One CTA per (tile, batch); each warp builds the bits of 16 query rows in
-// shared memory with shared atomics, then writes them out.
+//
+// Two launches:
+//   topk_bitmap_rows_kernel   one warp per query row (B * tiles * 128 rows):
+//                             shared-memory atomics build the row's bits,
+//                             then the row's words are written for every
+//                             causal block (rows past T get zeros)
+//   topk_block_list_kernel    one CTA per (tile, batch): OR of each block's
+//                             2 KB of bits, ballot-compacted into the list
+// No global atomics; the result is deterministic.
 #pragma once
 
+#include "mla.h"
 #include "ptx.cuh"
 
 namespace mla {
@@ -26,42 +34,51 @@ __host__ __device__ inline int64_t tri_index(int qt, int kb) {
 }
 
 __global__ void __launch_bounds__(32 * kPrepassWarps)
-topk_bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int nq,
-                   uint4* __restrict__ bitmap, int32_t* __restrict__ blocks) {
+topk_bitmap_rows_kernel(const int32_t* __restrict__ topk_idx, int B, int T, int k, int nq,
+                        uint4* __restrict__ bitmap) {
   extern __shared__ uint32_t psmem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kPrepassWarps + warp;  // over B * nq * 128
+  const int64_t rows_per_batch = static_cast<int64_t>(nq) * 128;
+  if (row >= static_cast<int64_t>(B) * rows_per_batch) return;
+  const int b = static_cast<int>(row / rows_per_batch);
+  const int s = static_cast<int>(row % rows_per_batch);
+  const int qt = s >> 7, r = s & 127;
+  const int nwords = (qt + 1) * 4;  // bits for keys [0, (qt+1)*128)
+  uint32_t* bits = psmem + warp * nq * 4;
+
+  for (int w = lane; w < nwords; w += 32) bits[w] = 0u;
+  __syncwarp();
+  if (s < T) {
+    const int32_t* idx = topk_idx + (static_cast<int64_t>(b) * T + s) * k;
+    for (int i = lane; i < k; i += 32) {
+      const int32_t t = __ldg(idx + i);
+      if (t >= 0 && t <= s) atomicOr(&bits[t >> 5], 1u << (t & 31));
+    }
+  }
+  __syncwarp();
+  uint32_t* bm = reinterpret_cast<uint32_t*>(bitmap + (b * tri_index(nq, 0) + tri_index(qt, 0)) * 128);
+  for (int w = lane; w < nwords; w += 32) bm[(static_cast<int64_t>(w >> 2) * 128 + r) * 4 + (w & 3)] = bits[w];
+}
+
+__global__ void __launch_bounds__(128)
+topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __restrict__ blocks) {
+  __shared__ uint32_t flags[MLA_MAX_T / 128];
   const int qt = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwords = (qt + 1) * 4;  // bits for keys [0, (qt+1)*128)
-  uint32_t* flags = psmem;                       // [nq] any-bit flag per key block
-  uint32_t* rowbits = psmem + nq + warp * nq * 4;  // this warp's row, [nq*4] words
-  for (int i = threadIdx.x; i < nq; i += blockDim.x) flags[i] = 0;
-  __syncthreads();
-
-  const int64_t tri_total = tri_index(nq, 0);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(bitmap + (b * tri_total + tri_index(qt, 0)) * 128);
-
-  for (int r = warp; r < 128; r += kPrepassWarps) {
-    const int s = qt * 128 + r;
-    for (int w = lane; w < nwords; w += 32) rowbits[w] = 0u;
-    __syncwarp();
-    if (s < T) {
-      const int32_t* idx = topk_idx + (static_cast<int64_t>(b) * T + s) * k;
-      for (int i = lane; i < k; i += 32) {
-        const int32_t t = __ldg(idx + i);
-        if (t >= 0 && t <= s) atomicOr(&rowbits[t >> 5], 1u << (t & 31));
-      }
+  const uint4* tile = bitmap + (b * tri_index(nq, 0) + tri_index(qt, 0)) * 128;
+  for (int kb = warp; kb <= qt; kb += 4) {
+    const uint4* blk = tile + static_cast<int64_t>(kb) * 128;
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = __ldg(blk + lane + 32 * i);
+      acc |= v.x | v.y | v.z | v.w;
     }
-    __syncwarp();
-    for (int w = lane; w < nwords; w += 32) {
-      const uint32_t v = rowbits[w];
-      const int kb = w >> 2;
-      bm[(static_cast<int64_t>(kb) * 128 + r) * 4 + (w & 3)] = v;
-      if (v) flags[kb] = 1u;
-    }
-    __syncwarp();
+    const bool any = __any_sync(0xffffffffu, acc != 0u);
+    if (lane == 0) flags[kb] = any ? 1u : 0u;
   }
   __syncthreads();
-
   if (warp == 0) {
     int32_t* out = blocks + (static_cast<int64_t>(b) * nq + qt) * (nq + 1);
     int count = 0;

@@ -85,6 +85,8 @@ def test_host_validation_before_any_device_work(lib):
     assert _attend(lib, _dims(wdtype=1)) == 1                  # e4m3 without scales
     assert _attend(lib, _dims(topk=0), {"tk": 16}) == 2        # top-k rows of width 0
     assert _attend(lib, _dims(), scale=float("nan")) == 2
+    assert _attend(lib, _dims(), scale=0.0) == 2
+    assert _attend(lib, _dims(), scale=-0.1) == 2
     assert _attend(lib, _dims(), {"q": 24}) == 6               # misaligned
     assert _attend(lib, _dims()) == 4                          # workspace missing
     assert _attend(lib, _dims(), ws=16, nbytes=100) == 4       # workspace too small
