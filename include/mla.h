@@ -52,7 +52,9 @@ typedef enum {
   MLA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than mla_workspace_bytes() */
   MLA_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
   MLA_ERR_ALIGN = 6,        /* a pointer is not 16-byte aligned */
-  MLA_ERR_DEVICE = 7        /* a kernel recorded a device-side error (see mla_device_status) */
+  MLA_ERR_DEVICE = 7,       /* a kernel recorded a device-side error (see mla_device_status) */
+  MLA_ERR_TOO_LARGE = 8     /* the problem needs more scratch than mla_attend_static's built-in
+                               MLA_STATIC_SCRATCH_BYTES */
 } mla_status;
 
 typedef enum {
@@ -130,6 +132,35 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent,
                 const void* W_o, const float* W_o_scale, const int32_t* topk_idx,
                 float scale, void* out, void* workspace, size_t ws_bytes,
                 mla_stream_t stream);
+
+/* mla_attend without a caller-supplied workspace (no counterpart on the
+ * pages: it exists for callers that cannot hand the library device memory).
+ *
+ * Some callers cannot call cudaMalloc: a plugin running inside a host
+ * framework that owns all device memory through its own pool and hands out
+ * no raw allocations, or a latency-critical path where cudaMalloc's implicit
+ * device synchronisation is not acceptable. This entry runs exactly the
+ * mla_attend computation, but its scratch (up-projected kv, selection
+ * bitmap, block lists) lives in one file-scope device array of
+ * MLA_STATIC_SCRATCH_BYTES that the library module holds on every GPU that
+ * loads it, from load until process exit. It allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - Arguments and layouts: as for mla_attend (minus workspace/ws_bytes).
+ *   - Limit: returns MLA_ERR_TOO_LARGE, before launching anything, when
+ *     mla_workspace_bytes(dims, MLA_ENTRY_ATTEND, topk_idx != NULL) exceeds
+ *     MLA_STATIC_SCRATCH_BYTES (e.g. B*T*H*512 bytes of kv alone).
+ *   - Set-up: the first call on a device (with that device current) looks
+ *     up the array's device address once (cudaGetSymbolAddress); make that
+ *     first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     previous call's contents; each call writes every scratch word it reads,
+ *     so nothing has to start at zero. Calls that overlap on the GPU (other
+ *     streams, other host threads) race on the array: order them. */
+#define MLA_STATIC_SCRATCH_BYTES (32u << 20)
+int mla_attend_static(const mla_dims* dims, const void* q, const void* kv_latent,
+                      const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
+                      const int32_t* topk_idx, float scale, void* attn_out,
+                      mla_stream_t stream);
 
 /* Human-readable text of a status code (static storage). */
 const char* mla_status_str(int status);

@@ -17,6 +17,7 @@ from .mla import (  # noqa: F401
     load_library,
     make_dims,
     mla_attend,
+    mla_attend_static,
     mla_device_status,
     mla_kv_upproject,
     mla_out_project,

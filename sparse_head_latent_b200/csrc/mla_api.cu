@@ -467,6 +467,7 @@ const char* mla_status_str(int status) {
     case MLA_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case MLA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
     case MLA_ERR_DEVICE: return "a kernel recorded a device-side error";
+    case MLA_ERR_TOO_LARGE: return "problem needs more scratch than the built-in MLA_STATIC_SCRATCH_BYTES";
     default: return "unknown status";
   }
 }
@@ -520,3 +521,57 @@ int mla_profile_end(float* ms_total, int* launches) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ built-in scratch entry point
+
+// Scratch of mla_attend_static for callers that cannot allocate device
+// memory. The module holds it on every GPU that loads the library.
+__device__ __align__(256) uint8_t g_mla_static_scratch[MLA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_mutex;
+std::vector<uint8_t*> g_static_scratch;  // device address of the array, per device (NULL: not looked up)
+
+// Device address of g_mla_static_scratch on the current device, looked up
+// once per device. In host code the array's name is only a host-side
+// stand-in, so kernels must be given this address instead.
+int static_scratch(uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (static_cast<int>(g_static_scratch.size()) <= dev) g_static_scratch.resize(dev + 1, nullptr);
+  if (g_static_scratch[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mla_static_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    g_static_scratch[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_static_scratch[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_attend_static(const mla_dims* dims, const void* q, const void* kv_latent, const void* k_pe,
+                                 const void* W_kvb, const float* W_kvb_scale, const int32_t* topk_idx, float scale,
+                                 void* attn_out, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!q || !kv_latent || !k_pe || !W_kvb || !attn_out || !fp8_scales_ok(dims, W_kvb_scale)) return MLA_ERR_NULL;
+  if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MLA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(attn_out) ||
+      !aligned16(W_kvb_scale) || !aligned16(topk_idx))
+    return MLA_ERR_ALIGN;
+  const WsLayout lay = ws_layout(*dims, MLA_ENTRY_ATTEND, topk_idx != nullptr);
+  if (lay.total > MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_TOO_LARGE;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != MLA_OK) return rc;
+  uint8_t* scratch = nullptr;
+  rc = static_scratch(&scratch);
+  if (rc != MLA_OK) return rc;
+  return run_attend(ds, *dims, lay, scratch, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, attn_out,
+                    reinterpret_cast<cudaStream_t>(stream));
+}

@@ -48,6 +48,8 @@ SIGNATURES = {
     "mla_out_project": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mla_prefill": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                    ctypes.c_float, _VP, _VP, _SZ, _VP]),
+    "mla_attend_static": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_float,
+                                         _VP, _VP]),
     "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int)]),
     "mla_profile_begin": (ctypes.c_int, []),
@@ -154,6 +156,27 @@ def mla_attend(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale
     _check("mla_attend", lib.mla_attend(ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb),
                                         _ptr(W_kvb_scale), _ptr(topk_idx), float(scale), _ptr(attn_out),
                                         _ptr(ws), nbytes, _stream(stream)))
+    return attn_out
+
+
+MLA_STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def mla_attend_static(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale=192 ** -0.5,
+                      attn_out=None, stream=None):
+    """mla_attend with the library's built-in scratch instead of a workspace,
+    for callers that cannot allocate device memory; problems whose scratch
+    exceeds MLA_STATIC_SCRATCH_BYTES are rejected (MlaError, status 8)."""
+    B, T, H, _ = q.shape
+    topk = 0 if topk_idx is None else topk_idx.shape[-1]
+    dims = make_dims(B, T, H, topk, _wtype(W_kvb))
+    if topk_idx is not None and topk_idx.dtype != torch.int32:
+        raise ValueError("topk_idx must be int32")
+    if attn_out is None:
+        attn_out = torch.empty(B, T, H, D_V, dtype=torch.bfloat16, device=q.device)
+    _check("mla_attend_static", load_library().mla_attend_static(
+        ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb), _ptr(W_kvb_scale), _ptr(topk_idx),
+        float(scale), _ptr(attn_out), _stream(stream)))
     return attn_out
 
 
