@@ -46,7 +46,8 @@ struct AttnSmem {
   static constexpr int V1 = 180224;        // stage 1
   static constexpr int BARS = 212992;
   static constexpr int NUM_BARS = 16;
-  static constexpr int BYTES = 1024 + BARS + NUM_BARS * 8 + 16;
+  static constexpr int BLIST = BARS + 256;  // active key-block ids of this tile (<= MLA_MAX_T / 128)
+  static constexpr int BYTES = 1024 + BLIST + (MLA_MAX_T / 128) * 4;
 };
 
 // Tensor-memory columns.
@@ -87,8 +88,13 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const int qt = p.nq - 1 - rem0 / (p.B * p.hgroup);
   const int rem = rem0 % (p.B * p.hgroup);
   const int b = rem / p.hgroup, h = hg * p.hgroup + rem % p.hgroup;
-  const int32_t* blist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.nq + qt) * (p.nq + 1) : nullptr;
-  const int n = blist ? blist[0] : qt + 1;
+  const int32_t* gblist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.nq + qt) * (p.nq + 1) : nullptr;
+  const int n = gblist ? gblist[0] : qt + 1;
+  // Key-block ids in shared memory (read by every role once per block).
+  int32_t* blist = gblist ? reinterpret_cast<int32_t*>(smem + AttnSmem::BLIST) : nullptr;
+  if (gblist) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) blist[i] = gblist[1 + i];
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQFull), 1);
@@ -132,7 +138,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       auto load_k = [&](int j) -> bool {
         const int ks = j & 1;
         if (!mbar_wait(bar(kBarKEmpty0 + ks), ((j >> 1) & 1) ^ 1, ab, kErrWaitMma)) return false;
-        const int t0 = (blist ? blist[1 + j] : j) * 128;
+        const int t0 = (blist ? blist[j] : j) * 128;
         const uint32_t dst = smem_u32(smem + (ks ? AttnSmem::K1 : AttnSmem::K0));
         const uint32_t fb = bar(kBarKFull0 + ks);
         mbar_arrive_expect_tx(fb, 3 * 16384);
@@ -147,7 +153,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (j + 1 < n && !(ok = load_k(j + 1))) break;
         const int vs = j & 1;
         if (!(ok = mbar_wait(bar(kBarVEmpty0 + vs), ((j >> 1) & 1) ^ 1, ab, kErrWaitMma))) break;
-        const int t0 = (blist ? blist[1 + j] : j) * 128;
+        const int t0 = (blist ? blist[j] : j) * 128;
         const uint32_t dst = smem_u32(smem + (vs ? AttnSmem::V1 : AttnSmem::V0));
         const uint32_t fb = bar(kBarVFull0 + vs);
         mbar_arrive_expect_tx(fb, 2 * 16384);
@@ -219,13 +225,15 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 domain) and sum
     bool ok = true;
 
+    // Selection words of this row, fetched one block ahead.
+    const uint4* bm_row = p.bitmap ? p.bitmap + (static_cast<int64_t>(b) * tri_total + tri_index(qt, 0)) * 128 + r
+                                   : nullptr;
+    uint4 bits_next = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu);
+    if (bm_row && n > 0) bits_next = __ldg(bm_row + static_cast<int64_t>(blist ? blist[0] : 0) * 128);
     for (int j = 0; j < n; ++j) {
-      const int kb = blist ? blist[1 + j] : j;
-      uint32_t bw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (p.bitmap) {
-        const uint4 v = __ldg(p.bitmap + (static_cast<int64_t>(b) * tri_total + tri_index(qt, kb)) * 128 + r);
-        bw[0] = v.x; bw[1] = v.y; bw[2] = v.z; bw[3] = v.w;
-      }
+      const int kb = blist ? blist[j] : j;
+      const uint32_t bw[4] = {bits_next.x, bits_next.y, bits_next.z, bits_next.w};
+      if (bm_row && j + 1 < n) bits_next = __ldg(bm_row + static_cast<int64_t>(blist ? blist[j + 1] : j + 1) * 128);
       const int st = j & 1;
       if (!(ok = warp_wait(bar(kBarSFull0 + st), (j >> 1) & 1, ab, kErrWaitMma))) break;
       tc_fence_after();

@@ -1,50 +1,64 @@
-// gemm.cuh -- persistent tcgen05 GEMM for sm_100a: C[M,N] = A[M,K] * B, bf16
-// operands, fp32 accumulation in tensor memory, bf16 output.
+// gemm2.cuh -- persistent tcgen05 GEMM on CTA pairs (cta_group::2) for sm_100a:
+// C[M,N] = A[M,K] * B, bf16 operands, fp32 accumulation in tensor memory,
+// bf16 output.
 //
-// Used for the W_kvb up-projection (A = latent [M, 512], B = W_kvb stored
-// [N, K] i.e. K-major) and for the output projection (A = attention output
-// [M, H*128], B = W_o stored [K, N] i.e. N-major).
+// A cluster of two CTAs on two SMs computes one 256 x 256 output tile with a
+// single M=256, N=256 UMMA per K step, issued by the leader CTA (rank 0):
+//   CTA r holds A rows [128r, 128r+128) and B columns [128r, 128r+128) of
+//   the tile (each CTA TMA-loads its own halves; nothing is multicast), and
+//   its tensor memory receives D rows [128r, 128r+128).
+// Per SM this moves (128 + 128) x K operand elements for a 128 x 256 share
+// of the output, a third less L2->SM traffic than a 128 x 256 tile with a
+// single CTA, which is what bounds the output projection.
 //
-// One CTA per SM, 192 threads:
-//   warp 0      TMA producer: A and B tiles into a STAGES-deep ring
-//   warp 1      tensor-memory allocator and UMMA issuer (one elected lane)
-//   warps 2..5  epilogue: tensor memory -> registers -> bf16 -> swizzled
-//               shared staging -> TMA store
-// Two 128 x BN fp32 accumulators in tensor memory let the epilogue of one
-// tile run under the main loop of the next.
+// Roles per CTA (192 threads), as in the single-CTA kernel:
+//   warp 0      TMA producer for this CTA's halves; completion is counted on
+//               the leader's full barrier
+//   warp 1      tensor-memory allocator (both CTAs, cta_group::2); UMMA
+//               issuer in the leader only; commits arrive on both CTAs
+//   warps 2..5  epilogue on this CTA's 128 rows; releases the accumulator
+//               by arriving on the leader's barrier
 #pragma once
 
 #include "ptx.cuh"
 
 namespace mla {
 
-template <int BN_, bool B_MN_MAJOR_>
-struct GemmCfg {
-  static constexpr int BM = 128;
-  static constexpr int BN = BN_;
-  static constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+template <bool B_MN_MAJOR_>
+struct Gemm2Cfg {
+  static constexpr int BM = 256;       // per CTA pair
+  static constexpr int BN = 256;       // per CTA pair
+  static constexpr int HM = 128;       // A rows per CTA
+  static constexpr int HN = 128;       // B columns per CTA
+  static constexpr int BK = 64;
   static constexpr bool B_MN_MAJOR = B_MN_MAJOR_;
-  static constexpr int STAGES = 4;
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = HM * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = HN * BK * 2;   // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_WARPS = 4;
-  static constexpr int EPI_BUF = 32 * 128;  // 32 rows x 64 bf16 columns
+  static constexpr int EPI_BUF = 32 * 128;
   static constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
   static constexpr int NUM_BARS = 2 * STAGES + 4;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + NUM_BARS * 8 + 16;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be a multiple of 64 in [64, 256]");
-  static_assert(2 * BN <= 512, "two accumulators must fit in tensor memory");
+  static constexpr uint32_t TMEM_COLS = 512;   // two 256-column accumulators
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// Spin for about `ns` nanoseconds (used only to let in-flight copies land on
+// the abort path, where this CTA cannot observe the leader's barrier).
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) {
+  }
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
-gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int* err) {
-  constexpr int BM = Cfg::BM, BN = Cfg::BN, BK = Cfg::BK, S = Cfg::STAGES;
+gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int* err) {
+  constexpr int BK = Cfg::BK, S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi = smem + S * Cfg::STAGE_BYTES;
@@ -58,6 +72,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const uint32_t acce0 = smem_u32(bars + 2 * S + 2);
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -66,7 +82,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
-      mbar_init(acce0 + 8 * a, Cfg::EPI_WARPS);
+      mbar_init(acce0 + 8 * a, 2 * Cfg::EPI_WARPS);  // epilogue warps of both CTAs
     }
     *abort_word = 0;
     fence_barrier_init();
@@ -77,27 +93,32 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     prefetch_tmap(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const Abort ab{abort_word, err};
 
-  const int num_m = (M + BM - 1) / BM;
-  const int num_n = N / BN;
+  const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
+  const int num_n = N / Cfg::BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = K / BK;
+  const int pair = static_cast<int>(blockIdx.x) >> 1;
+  const int num_pairs = static_cast<int>(gridDim.x) >> 1;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer (this CTA's halves)
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         const int mt = tile % num_m, nt = tile / num_m;
+        const int arow = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM;
+        const int bcol = nt * Cfg::BN + static_cast<int>(rank) * Cfg::HN;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -105,31 +126,28 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ok = false;
             break;
           }
-          const uint32_t full = full0 + 8 * s;
+          const uint32_t full_leader = mapa_shared(full0 + 8 * s, 0);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * Cfg::STAGE_BYTES);
           const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t sb = sa + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(full, Cfg::STAGE_BYTES);
-          tma_load_2d(sa, &tmA, full, kb * BK, mt * BM);
+          tma_load_2d_pair(sa, &tmA, full_leader, kb * BK, arow);
           if constexpr (!Cfg::B_MN_MAJOR) {
-            tma_load_2d(sb, &tmB, full, kb * BK, nt * BN);
+            tma_load_2d_pair(sb, &tmB, full_leader, kb * BK, bcol);
           } else {
-#pragma unroll
-            for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * (BK * 128), &tmB, full, nt * BN + c * 64, kb * BK);
+            tma_load_2d_pair(sb, &tmB, full_leader, bcol, kb * BK);
+            tma_load_2d_pair(sb + BK * 128, &tmB, full_leader, bcol + 64, kb * BK);
           }
         }
       }
-      if (!ok) {
-        // Let every load already issued land before the CTA exits.
-        for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait_drain(full0 + 8 * (i % S), (i / S) & 1);
-      }
+      if (!ok) spin_ns(2000000);  // let issued loads land before the CTA can exit
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- UMMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, Cfg::B_MN_MAJOR ? 1 : 0);
+    if (lane == 0 && leader) {
+      // ---------------- UMMA issuer (leader CTA only)
+      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, 0, Cfg::B_MN_MAJOR ? 1 : 0);
       int it = 0, t = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++t) {
         const int a = t & 1;
         const uint32_t aph = (t >> 1) & 1;
         if (!mbar_wait(acce0 + 8 * a, aph ^ 1, ab, kErrWaitEpilogue)) {
@@ -137,7 +155,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + a * BN;
+        const uint32_t d = tmem_base + a * 256;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -153,33 +171,33 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint64_t adesc = smem_desc_sw128(sa + k * 32, 16, 1024);
             const uint64_t bdesc = Cfg::B_MN_MAJOR ? smem_desc_sw128(sb + k * 16 * 128, BK * 128, 1024)
                                                    : smem_desc_sw128(sb + k * 32, 16, 1024);
-            umma_ss(d, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_ss_pair(d, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(empty0 + 8 * s);
+          umma_commit_pair(empty0 + 8 * s, 0x3);
         }
         if (!ok) break;
-        umma_commit(accf0 + 8 * a);
+        umma_commit_pair(accf0 + 8 * a, 0x3);
       }
       if (!ok && it > 0) {
-        const int i = it - 1;  // the last commit covers every earlier MMA
+        const int i = it - 1;
         mbar_wait_drain(empty0 + 8 * (i % S), (i / S) & 1);
       }
     }
   } else {
-    // ---------------- epilogue warps
-    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+    // ---------------- epilogue warps: this CTA's 128 rows of the tile
+    const int q = warp & 3;
     uint8_t* bufs = epi + (warp - 2) * 2 * Cfg::EPI_BUF;
     int t = 0, nbuf = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
       const int mt = tile % num_m, nt = tile / num_m;
       const int a = t & 1;
       const uint32_t aph = (t >> 1) & 1;
       if (!warp_wait(accf0 + 8 * a, aph, ab, kErrWaitMma)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
-      const int row0 = mt * BM + q * 32;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * 256;
+      const int row0 = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM + q * 32;
 #pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
+      for (int c = 0; c < Cfg::BN / 64; ++c) {
         uint32_t r0[32], r1[32];
         tmem_ld32x2(tb + c * 64, tb + c * 64 + 32, r0, r1);
         uint8_t* buf = bufs + (nbuf & 1) * Cfg::EPI_BUF;
@@ -207,22 +225,23 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && row0 < M) {
-          tma_store_2d(&tmC, smem_u32(buf), nt * BN + c * 64, row0);
+          tma_store_2d(&tmC, smem_u32(buf), nt * Cfg::BN + c * 64, row0);
           bulk_commit_group();
         }
         ++nbuf;
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce0 + 8 * a);
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(acce0 + 8 * a, 0));
     }
     if (lane == 0) bulk_wait_group<0>();
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the leader's UMMAs read the peer's shared memory until here
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
 }
 
 }  // namespace mla

@@ -15,7 +15,7 @@
 #include "../../include/mla.h"
 #include "attn.cuh"
 #include "dequant.cuh"
-#include "gemm.cuh"
+#include "gemm2.cuh"
 #include "prepass.cuh"
 #include "ptx.cuh"
 
@@ -24,11 +24,9 @@ __device__ int g_mla_device_error;
 
 namespace {
 
-using mla::GemmCfg;
-
 constexpr int kDn = 128, kDr = 64, kDv = 128, kL = 512, kD = 7168;
-using GemmKvb = GemmCfg<256, false>;  // latent x W_kvb^T  (B stored [N, K])
-using GemmWo = GemmCfg<256, true>;    // attn x W_o         (B stored [K, N])
+using Gemm2Kvb = mla::Gemm2Cfg<false>;  // latent x W_kvb^T  (B stored [N, K])
+using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N])
 
 // ------------------------------------------------------------------ device state
 
@@ -36,8 +34,28 @@ struct DeviceState {
   bool ready = false;
   int status = MLA_OK;
   int sms = 0;
+  int pairs_kvb = 0;   // CTA pairs of the pair GEMMs that fit on the device at once
+  int pairs_wo = 0;
   int* err = nullptr;  // address of g_mla_device_error on this device
 };
+
+template <class Kernel>
+int max_pairs(Kernel k, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) return 0;
+  return n;
+}
 
 std::mutex g_mutex;
 std::vector<DeviceState> g_devices;
@@ -66,10 +84,15 @@ int device_state(DeviceState** out) {
       st.sms = prop.multiProcessorCount;
       bool ok = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err), g_mla_device_error) == cudaSuccess;
       ok = ok && cudaMemset(st.err, 0, sizeof(int)) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc_kernel<GemmKvb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      GemmKvb::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc_kernel<GemmWo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      GemmWo::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Gemm2Kvb::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Gemm2Wo::SMEM_BYTES) == cudaSuccess;
+      if (ok) {
+        st.pairs_kvb = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, Gemm2Kvb::SMEM_BYTES);
+        st.pairs_wo = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, Gemm2Wo::SMEM_BYTES);
+        ok = st.pairs_kvb > 0 && st.pairs_wo > 0;
+      }
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AttnSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::topk_bitmap_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -224,20 +247,38 @@ int launch_dequant(const DeviceState* ds, const void* codes, const float* scale,
   });
 }
 
+template <class Cfg>
+int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M,
+                     int N, int K, int* err, int cls, cudaStream_t st) {
+  const int tiles = ((M + Cfg::BM - 1) / Cfg::BM) * (N / Cfg::BN);
+  const int pairs = tiles < pairs_max ? tiles : pairs_max;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+  const int rc = timed_launch(
+      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, err); });
+  return le != cudaSuccess ? MLA_ERR_CUDA : rc;
+}
+
 int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const void* wkvb, void* kvh,
                     cudaStream_t st) {
   const int N = H * (kDn + kDv), K = kL;
   CUtensorMap ta, tb, tc;
   if (!map_2d(&ta, lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, 128) ||
-      !map_2d(&tb, wkvb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, GemmKvb::BN) ||
+      !map_2d(&tb, wkvb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, Gemm2Kvb::HN) ||
       !map_2d(&tc, kvh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
     return MLA_ERR_CUDA;
-  const int tiles = ((M + 127) / 128) * (N / GemmKvb::BN);
-  const int grid = tiles < ds->sms ? tiles : ds->sms;
-  return timed_launch(2, st, [&] {
-    mla::gemm_bf16_tc_kernel<GemmKvb><<<grid, GemmKvb::THREADS, GemmKvb::SMEM_BYTES, st>>>(ta, tb, tc, M, N, K,
-                                                                                         ds->err);
-  });
+  return launch_gemm_pair<Gemm2Kvb>(ds->pairs_kvb, ta, tb, tc, M, N, K, ds->err, 2, st);
 }
 
 int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const void* wo, void* out,
@@ -248,12 +289,7 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
       !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64) ||
       !map_2d(&tc, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
     return MLA_ERR_CUDA;
-  const int tiles = ((M + 127) / 128) * (N / GemmWo::BN);
-  const int grid = tiles < ds->sms ? tiles : ds->sms;
-  return timed_launch(4, st, [&] {
-    mla::gemm_bf16_tc_kernel<GemmWo><<<grid, GemmWo::THREADS, GemmWo::SMEM_BYTES, st>>>(ta, tb, tc, M, N, K,
-                                                                                      ds->err);
-  });
+  return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st);
 }
 
 int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks,
