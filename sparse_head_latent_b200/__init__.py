@@ -13,6 +13,7 @@ from .mla import (  # noqa: F401
     MLA_ENTRY_PREFILL,
     MlaDims,
     MlaError,
+    PrefillPipeline,
     library_path,
     load_library,
     make_dims,

@@ -6,8 +6,13 @@
 //   S   = q_h . [k_nope_h | k_pe]^T              (UMMA, K = 192, S in tensor memory)
 //   S   = -inf where bit(s, t) = 0                (top-k + causal selection)
 //   m,l = running max / sum of exp2(S*scale*log2e - m) per query row (fp32)
-//   O  += P . v_h                                 (UMMA, P bf16 in tensor memory, O in tensor memory)
+//   O  += P . v_h                                 (UMMA, P f16 in tensor memory, O in tensor memory)
+//   l  += P . 1                                   (UMMA against a constant block of ones)
 //   attn[b, s, h, :] = O / l                      (bf16)
+// P is exp2 of the scaled scores, computed two at a time in f16
+// (ex2.approx.f16x2); v is stored as f16 by the up-projection, so PV is an
+// f16 x f16 UMMA with fp32 accumulation and the row sums come from the
+// tensor core, never from the softmax warps.
 // Neither the [T, T] scores nor a float mask is ever materialised: the
 // selection arrives as one bit per causal (query, key) pair.
 //
@@ -18,9 +23,9 @@
 //               next block before PV of the current one so the tensor core
 //               works while the softmax runs
 //   warps 2..5  softmax: one query row per thread (tensor-memory lane)
-// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384), P [384,448)
-// (P: 128 bf16 per row packed in 64 columns; the PV UMMA reads it as its A
-// operand, so P never touches shared memory).
+// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384), l [384,400),
+// P [416,480) (P: 128 f16 per row packed in 64 columns; the PV UMMA reads it
+// as its A operand, so P never touches shared memory).
 #pragma once
 
 #include "prepass.cuh"
@@ -44,14 +49,15 @@ struct AttnSmem {
   static constexpr int K1 = 98304;         // stage 1
   static constexpr int V0 = 147456;        // stage 0: 2 x [128 keys x 64 dv]
   static constexpr int V1 = 180224;        // stage 1
-  static constexpr int BARS = 212992;
+  static constexpr int ONES = 212992;      // [16 x 128] f16 ones (row-sum operand)
+  static constexpr int BARS = 217088;
   static constexpr int NUM_BARS = 16;
   static constexpr int BLIST = BARS + 256;  // active key-block ids of this tile (<= MLA_MAX_T / 128)
   static constexpr int BYTES = 1024 + BLIST + (MLA_MAX_T / 128) * 4;
 };
 
 // Tensor-memory columns.
-constexpr uint32_t kTmemS0 = 0, kTmemO = 256, kTmemP = 384;
+constexpr uint32_t kTmemS0 = 0, kTmemO = 256, kTmemL = 384, kTmemP = 416;
 
 // Barrier slots.
 enum : int {
@@ -62,6 +68,31 @@ enum : int {
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (x0, x1) <- (x0 * c + b, x1 * c + b) as one packed f32x2 FMA.
+__device__ __forceinline__ void fma2_scalar(float& x0, float& x1, float c, float b) {
+  asm("{\n\t.reg .b64 t, u, v;\n\t"
+      "mov.b64 t, {%0, %1};\n\t"
+      "mov.b64 u, {%2, %2};\n\t"
+      "mov.b64 v, {%3, %3};\n\t"
+      "fma.rn.f32x2 t, t, u, v;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(c), "f"(b));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2 of two f16 values at once (MUFU ex2.approx on an f16 pair).
+__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
@@ -94,6 +125,11 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   int32_t* blist = gblist ? reinterpret_cast<int32_t*>(smem + AttnSmem::BLIST) : nullptr;
   if (gblist) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) blist[i] = gblist[1 + i];
+  }
+  {
+    uint4* ones = reinterpret_cast<uint4*>(smem + AttnSmem::ONES);
+    for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x) ones[i] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    fence_proxy_async_smem();  // read by the tensor core through a descriptor
   }
 
   if (threadIdx.x == 0) {
@@ -171,7 +207,9 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (lane == 0 && n > 0) {
       // ---------------- UMMA issuer
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, 0, 1);
+      constexpr uint32_t idesc_l = idesc_f16_f32(128, 16, 0, 0);
+      const uint32_t sOnes = smem_u32(smem + AttnSmem::ONES);
       bool ok = mbar_wait(bar(kBarQFull), 0, ab, kErrWaitTma);
       int issued = 0;
       auto issue_qk = [&](int j) -> bool {
@@ -205,6 +243,12 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           const uint64_t bdesc = smem_desc_sw128(sV + k * 2048, 16384, 1024);
           umma_ts(tmem + kTmemO, tmem + kTmemP + k * 8, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
         }
+        // Row sums: l += P . ones (every one of the 16 columns gets the sum).
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t odesc = smem_desc_sw128(sOnes + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024);
+          umma_ts(tmem + kTmemL, tmem + kTmemP + k * 8, odesc, idesc_l, (j > 0 || k > 0) ? 1u : 0u);
+        }
         ++issued;
         umma_commit(bar(kBarVEmpty0 + vs));
         umma_commit(bar(kBarPvDone));
@@ -222,7 +266,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int64_t tri_total = tri_index(p.nq, 0);
     const float c = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 domain) and sum
+    float m_run = -INFINITY;  // running max (scaled log2 domain); the sums live in tensor memory
     bool ok = true;
 
     // Selection words of this row, fetched one block ahead.
@@ -262,16 +306,21 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
         for (int i = 0; i < 128; ++i) x[i] = ((bw[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
       }
-      // Row max with 8 independent chains.
+      // Row max: 8 independent chains of 3-input max.
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = x[i];
+      for (int i = 0; i < 8; ++i) mx[i] = max3(x[i], x[8 + i], x[16 + i]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], x[i]);
-      const float mblk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+      for (int k0 = 24; k0 < 120; k0 += 16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], x[k0 + i], x[k0 + 8 + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], x[120 + i]);
+      const float mblk = fmaxf(max3(mx[0], mx[1], mx[2]), max3(mx[3], max3(mx[4], mx[5], mx[6]), mx[7])) * c;
       // Lazy rescaling: keep the running max unless the block max exceeds it
-      // by more than 8 (a factor of 256), so O is rarely touched.
+      // by more than 8 (a factor of 256), so O and l are rarely touched and P
+      // stays below 2^8 (well inside f16).
       const float m_new = fmaxf(m_run, mblk);
       const bool resc = (m_new - m_run) > 8.f;
       float alpha = 1.f;
@@ -279,25 +328,24 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         alpha = ex2_approx(m_run - m_new);
         m_run = m_new;
       }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float sm[8];
+      const float nb = (m_run == -INFINITY) ? 0.f : -m_run;
+      // P = exp2(S*c - m): the argument in fp32 (packed FMA), the exp2 on f16
+      // pairs; masked entries are -inf and give 0.
+      uint32_t pk[64];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sm[i] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        x[i] = ex2_approx(fmaf(x[i], c, -base));
-        sm[i & 7] += x[i];
+      for (int i = 0; i < 64; ++i) {
+        fma2_scalar(x[2 * i], x[2 * i + 1], c, nb);
+        pk[i] = ex2_f16x2(pack_f16x2(x[2 * i], x[2 * i + 1]));
       }
-      l_run = l_run * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
 
-      // PV of the previous block must be complete before O is rescaled and
-      // before P is overwritten.
+      // PV of the previous block must be complete before O and l are
+      // rescaled and before P is overwritten.
       if (j >= 1) {
         if (!(ok = warp_wait(bar(kBarPvDone), (j - 1) & 1, ab, kErrWaitMma))) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 32) {
+          for (int c0 = 0; c0 < 160; c0 += 32) {  // O (128 columns), then l (16) and 16 spare
             uint32_t o[32];
             tmem_ld32(trow + kTmemO + c0, o);
 #pragma unroll
@@ -306,15 +354,12 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           }
         }
       }
-      // P (bf16 pairs) into tensor memory, row r = lane r.
+      // P (f16 pairs) into tensor memory, row r = lane r.
       {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-        tmem_st32(trow + kTmemP, pk);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(x[64 + 2 * i], x[64 + 2 * i + 1]);
-        tmem_st32(trow + kTmemP + 32, pk);
+        uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+        uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+        tmem_st32(trow + kTmemP, p0);
+        tmem_st32(trow + kTmemP + 32, p1);
       }
       tc_fence_before();
       __syncwarp();
@@ -327,7 +372,10 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         ok = warp_wait(bar(kBarPvDone), (n - 1) & 1, ab, kErrWaitMma);
         if (ok) {
           tc_fence_after();
-          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          uint32_t lv[32];
+          tmem_ld32(trow + kTmemL, lv);
+          const float l_row = __uint_as_float(lv[0]);
+          const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
 #pragma unroll 1
           for (int c0 = 0; c0 < 128; c0 += 64) {
             uint32_t a0[32], a1[32];

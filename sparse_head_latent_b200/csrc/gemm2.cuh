@@ -24,7 +24,10 @@
 
 namespace mla {
 
-template <bool B_MN_MAJOR_>
+// V_F16: the output columns [128, 256) of every 256-column tile are stored
+// as f16 instead of bf16. With N = H*256 that is the v half of each head of
+// the up-projection, which the attention kernel consumes as f16.
+template <bool B_MN_MAJOR_, bool V_F16_ = false>
 struct Gemm2Cfg {
   static constexpr int BM = 256;       // per CTA pair
   static constexpr int BN = 256;       // per CTA pair
@@ -32,6 +35,7 @@ struct Gemm2Cfg {
   static constexpr int HN = 128;       // B columns per CTA
   static constexpr int BK = 64;
   static constexpr bool B_MN_MAJOR = B_MN_MAJOR_;
+  static constexpr bool V_F16 = V_F16_;
   static constexpr int STAGES = 6;
   static constexpr int A_BYTES = HM * BK * 2;   // 16 KB
   static constexpr int B_BYTES = HN * BK * 2;   // 16 KB
@@ -204,23 +208,25 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
         uint8_t* rowp = buf + lane * 128;
+        const bool f16 = Cfg::V_F16 && c >= 2;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r0[8 * j + 0]), __uint_as_float(r0[8 * j + 1]));
-          v.y = pack_bf16x2(__uint_as_float(r0[8 * j + 2]), __uint_as_float(r0[8 * j + 3]));
-          v.z = pack_bf16x2(__uint_as_float(r0[8 * j + 4]), __uint_as_float(r0[8 * j + 5]));
-          v.w = pack_bf16x2(__uint_as_float(r0[8 * j + 6]), __uint_as_float(r0[8 * j + 7]));
-          *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = v;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r1[8 * j + 0]), __uint_as_float(r1[8 * j + 1]));
-          v.y = pack_bf16x2(__uint_as_float(r1[8 * j + 2]), __uint_as_float(r1[8 * j + 3]));
-          v.z = pack_bf16x2(__uint_as_float(r1[8 * j + 4]), __uint_as_float(r1[8 * j + 5]));
-          v.w = pack_bf16x2(__uint_as_float(r1[8 * j + 6]), __uint_as_float(r1[8 * j + 7]));
-          *reinterpret_cast<uint4*>(rowp + (((j + 4) ^ (lane & 7)) << 4)) = v;
+          const float* f0 = reinterpret_cast<const float*>(r0) + 8 * j;
+          const float* f1 = reinterpret_cast<const float*>(r1) + 8 * j;
+          uint4 v0, v1;
+          if (f16) {
+            v0 = make_uint4(pack_f16x2(f0[0], f0[1]), pack_f16x2(f0[2], f0[3]), pack_f16x2(f0[4], f0[5]),
+                            pack_f16x2(f0[6], f0[7]));
+            v1 = make_uint4(pack_f16x2(f1[0], f1[1]), pack_f16x2(f1[2], f1[3]), pack_f16x2(f1[4], f1[5]),
+                            pack_f16x2(f1[6], f1[7]));
+          } else {
+            v0 = make_uint4(pack_bf16x2(f0[0], f0[1]), pack_bf16x2(f0[2], f0[3]), pack_bf16x2(f0[4], f0[5]),
+                            pack_bf16x2(f0[6], f0[7]));
+            v1 = make_uint4(pack_bf16x2(f1[0], f1[1]), pack_bf16x2(f1[2], f1[3]), pack_bf16x2(f1[4], f1[5]),
+                            pack_bf16x2(f1[6], f1[7]));
+          }
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = v0;
+          *reinterpret_cast<uint4*>(rowp + (((j + 4) ^ (lane & 7)) << 4)) = v1;
         }
         fence_proxy_async_smem();
         __syncwarp();

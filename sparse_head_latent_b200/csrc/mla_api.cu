@@ -26,6 +26,7 @@ namespace {
 
 constexpr int kDn = 128, kDr = 64, kDv = 128, kL = 512, kD = 7168;
 using Gemm2Kvb = mla::Gemm2Cfg<false>;  // latent x W_kvb^T  (B stored [N, K])
+using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as f16 for the attention
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N])
 
 // ------------------------------------------------------------------ device state
@@ -88,6 +89,8 @@ int device_state(DeviceState** out) {
                                       Gemm2Kvb::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       Gemm2Wo::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2KvbAttn>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2KvbAttn::SMEM_BYTES) == cudaSuccess;
       if (ok) {
         st.pairs_kvb = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, Gemm2Kvb::SMEM_BYTES);
         st.pairs_wo = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, Gemm2Wo::SMEM_BYTES);
@@ -270,7 +273,8 @@ int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb
   return le != cudaSuccess ? MLA_ERR_CUDA : rc;
 }
 
-int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const void* wkvb, void* kvh,
+// v_f16: store the v half of every head as f16 (the attention path's kvh).
+int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const void* wkvb, void* kvh, bool v_f16,
                     cudaStream_t st) {
   const int N = H * (kDn + kDv), K = kL;
   CUtensorMap ta, tb, tc;
@@ -278,6 +282,7 @@ int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const 
       !map_2d(&tb, wkvb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, Gemm2Kvb::HN) ||
       !map_2d(&tc, kvh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
     return MLA_ERR_CUDA;
+  if (v_f16) return launch_gemm_pair<Gemm2KvbAttn>(ds->pairs_kvb, ta, tb, tc, M, N, K, ds->err, 2, st);
   return launch_gemm_pair<Gemm2Kvb>(ds->pairs_kvb, ta, tb, tc, M, N, K, ds->err, 2, st);
 }
 
@@ -362,7 +367,7 @@ int begin_call(const mla_dims* dims, int entry, bool has_topk, void* ws, size_t 
 // Up-projection into kvh; dequantises W_kvb into the workspace first when
 // it is stored as e4m3.
 int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* lat,
-                  const void* W_kvb, const float* W_kvb_scale, void* kvh, cudaStream_t st) {
+                  const void* W_kvb, const float* W_kvb_scale, void* kvh, bool v_f16, cudaStream_t st) {
   const void* wk = W_kvb;
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
     void* dq = ws_at(ws, lay.wkvb);
@@ -370,14 +375,14 @@ int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay,
     if (rc != MLA_OK) return rc;
     wk = dq;
   }
-  return launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, st);
+  return launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, v_f16, st);
 }
 
 int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* q,
                const void* lat, const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
                const int32_t* topk_idx, float scale, void* attn, cudaStream_t st) {
   void* kvh = ws_at(ws, lay.kvh);
-  int rc = run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, st);
+  int rc = run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, /*v_f16=*/true, st);
   if (rc != MLA_OK) return rc;
   void* bitmap = nullptr;
   void* blocks = nullptr;
@@ -426,7 +431,7 @@ int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_
   rc = begin_call(dims, MLA_ENTRY_KV_UPPROJECT, false, workspace, ws_bytes, &ds, &lay);
   if (rc != MLA_OK) return rc;
   if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
-  return run_upproject(ds, *dims, lay, workspace, kv_latent, W_kvb, W_kvb_scale, kvh_out,
+  return run_upproject(ds, *dims, lay, workspace, kv_latent, W_kvb, W_kvb_scale, kvh_out, /*v_f16=*/false,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -232,3 +232,67 @@ def mla_profile_end():
     n = (ctypes.c_int * MLA_PROFILE_CLASSES)()
     _check("mla_profile_end", load_library().mla_profile_end(ms, n))
     return {PROFILE_CLASS_NAMES[i]: (float(ms[i]), int(n[i])) for i in range(MLA_PROFILE_CLASSES)}
+
+
+class PrefillPipeline:
+    """mla_prefill over a stream of host batches, with the copies overlapped.
+
+    For batch i the host inputs (pinned CPU tensors) are copied to the device
+    on a copy stream while the kernels of batch i-1 run on the compute stream
+    and the output of batch i-2 is copied back on a third stream. Two device
+    buffer sets alternate; the weights stay resident. Every kernel is the C
+    ABI's; this class only orders copies and launches with CUDA events.
+    """
+
+    _INPUTS = ("q", "kv_latent", "k_pe", "topk_idx")
+
+    def __init__(self, B, T, H, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk=None,
+                 scale=192 ** -0.5, device=None):
+        dev = torch.device(device) if device is not None else W_o.device
+        self.dev, self.scale = dev, float(scale)
+        self.w = dict(W_kvb=W_kvb, W_o=W_o, W_kvb_scale=W_kvb_scale, W_o_scale=W_o_scale)
+        shapes = {"q": ((B, T, H, D_NOPE + D_ROPE), torch.bfloat16), "kv_latent": ((B, T, D_LATENT), torch.bfloat16),
+                  "k_pe": ((B, T, D_ROPE), torch.bfloat16)}
+        if topk is not None:
+            shapes["topk_idx"] = ((B, T, int(topk)), torch.int32)
+        self.slots = [{k: torch.empty(s, dtype=d, device=dev) for k, (s, d) in shapes.items()} for _ in range(2)]
+        for sl in self.slots:
+            sl["out"] = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=dev)
+        dims = make_dims(B, T, H, 0 if topk is None else topk, _wtype(W_kvb))
+        self.ws = torch.empty(max(1, mla_workspace_bytes(dims, MLA_ENTRY_PREFILL, topk is not None)),
+                              dtype=torch.uint8, device=dev)
+        self.h2d, self.comp, self.d2h = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.ev_in, self.ev_done, self.ev_out = ev(), ev(), ev()
+        self.used = [False, False]
+        self.i = 0
+
+    def submit(self, host_inputs: dict, host_out: torch.Tensor):
+        """Queues one batch: host_inputs maps q, kv_latent, k_pe (and topk_idx)
+        to pinned CPU tensors; the result lands in the pinned host_out."""
+        k = self.i & 1
+        sl = self.slots[k]
+        with torch.cuda.stream(self.h2d):
+            if self.used[k]:
+                self.h2d.wait_event(self.ev_done[k])  # the kernels that read this slot are done
+            for name in self._INPUTS:
+                if name in sl:
+                    sl[name].copy_(host_inputs[name], non_blocking=True)
+            self.ev_in[k].record(self.h2d)
+        self.comp.wait_event(self.ev_in[k])
+        if self.used[k]:
+            self.comp.wait_event(self.ev_out[k])  # the previous output of this slot has been copied out
+        mla_prefill(sl["q"], sl["kv_latent"], sl["k_pe"], self.w["W_kvb"], self.w["W_o"], self.w["W_kvb_scale"],
+                    self.w["W_o_scale"], topk_idx=sl.get("topk_idx"), scale=self.scale, out=sl["out"],
+                    workspace=self.ws, stream=self.comp)
+        self.ev_done[k].record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.ev_done[k])
+            host_out.copy_(sl["out"], non_blocking=True)
+            self.ev_out[k].record(self.d2h)
+        self.used[k] = True
+        self.i += 1
+
+    def synchronize(self):
+        for s in (self.h2d, self.comp, self.d2h):
+            s.synchronize()
