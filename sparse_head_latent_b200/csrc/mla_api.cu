@@ -309,7 +309,7 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
         topk, d.B, d.T, d.topk, nq, static_cast<uint4*>(bitmap));
   });
   if (rc != MLA_OK) return rc;
-  dim3 grid(nq, d.B);
+  dim3 grid((nq + 1) / 2, d.B);
   return timed_launch(0, st, [&] {
     mla::topk_block_list_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4*>(bitmap), nq,
                                                       static_cast<int32_t*>(blocks));
@@ -328,6 +328,7 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.T = d.T;
   p.H = d.H;
   p.nq = (d.T + 127) / 128;
+  p.npairs = (p.nq + 1) / 2;
   // Heads per scheduling group: the largest of 8, 4, 2, 1 that divides H and
   // keeps the group's K/V (T x 512 bytes per head and batch) near 48 MB or less.
   p.hgroup = 1;
@@ -342,9 +343,9 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.blocks = static_cast<const int32_t*>(blocks);
   p.attn = static_cast<__nv_bfloat16*>(attn);
   p.err = ds->err;
-  const int64_t grid = static_cast<int64_t>(d.B) * p.nq * d.H;
+  const int64_t grid = static_cast<int64_t>(d.B) * p.npairs * d.H;
   return timed_launch(3, st, [&] {
-    mla::sparse_mla_attn_kernel<<<static_cast<unsigned>(grid), 192, mla::AttnSmem::BYTES, st>>>(tq, tkv, tpe, p);
+    mla::sparse_mla_attn_kernel<<<static_cast<unsigned>(grid), mla::kAttnThreads, mla::AttnSmem::BYTES, st>>>(tq, tkv, tpe, p);
   });
 }
 

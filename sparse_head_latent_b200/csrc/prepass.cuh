@@ -9,16 +9,19 @@
 //
 // Layout (per batch b, 128-query tile qt, 128-key block kb <= qt):
 //   bitmap[b][qt*(qt+1)/2 + kb][row 0..127][4 x u32]   (bit c of the 128 = key kb*128 + c)
-//   blocks[b][qt][0] = number of key blocks with any bit set for the tile,
-//   blocks[b][qt][1 + i] = their indices, ascending.
+//   blocks[b][pair][0] = number of key blocks with any bit set for either
+//   query tile of the pair (tiles 2*pair and 2*pair+1, which the attention
+//   kernel processes together), blocks[b][pair][1 + i] = their indices,
+//   ascending.
 //
 // Two launches:
 //   topk_bitmap_rows_kernel   one warp per query row (B * tiles * 128 rows):
 //                             shared-memory atomics build the row's bits,
 //                             then the row's words are written for every
 //                             causal block (rows past T get zeros)
-//   topk_block_list_kernel    one CTA per (tile, batch): OR of each block's
-//                             2 KB of bits, ballot-compacted into the list
+//   topk_block_list_kernel    one CTA per (tile pair, batch): OR of each
+//                             block's bits over both tiles, ballot-compacted
+//                             into the pair's list
 // No global atomics; the result is deterministic.
 #pragma once
 
@@ -64,27 +67,31 @@ topk_bitmap_rows_kernel(const int32_t* __restrict__ topk_idx, int B, int T, int 
 __global__ void __launch_bounds__(128)
 topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __restrict__ blocks) {
   __shared__ uint32_t flags[MLA_MAX_T / 128];
-  const int qt = blockIdx.x, b = blockIdx.y;
+  const int pair = blockIdx.x, b = blockIdx.y;
+  const int qa = 2 * pair, qb = 2 * pair + 1;
+  const int last = qb < nq ? qb : qa;  // highest key block either tile can see
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint4* tile = bitmap + (b * tri_index(nq, 0) + tri_index(qt, 0)) * 128;
-  for (int kb = warp; kb <= qt; kb += 4) {
-    const uint4* blk = tile + static_cast<int64_t>(kb) * 128;
+  for (int kb = warp; kb <= last; kb += 4) {
     uint32_t acc = 0;
+    for (int qt = qa; qt <= last; ++qt) {
+      if (kb > qt) continue;  // outside this tile's causal triangle
+      const uint4* blk = bitmap + (b * tri_index(nq, 0) + tri_index(qt, kb)) * 128;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = __ldg(blk + lane + 32 * i);
-      acc |= v.x | v.y | v.z | v.w;
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(blk + lane + 32 * i);
+        acc |= v.x | v.y | v.z | v.w;
+      }
     }
     const bool any = __any_sync(0xffffffffu, acc != 0u);
     if (lane == 0) flags[kb] = any ? 1u : 0u;
   }
   __syncthreads();
   if (warp == 0) {
-    int32_t* out = blocks + (static_cast<int64_t>(b) * nq + qt) * (nq + 1);
+    int32_t* out = blocks + (static_cast<int64_t>(b) * nq + pair) * (nq + 1);
     int count = 0;
-    for (int base = 0; base <= qt; base += 32) {
+    for (int base = 0; base <= last; base += 32) {
       const int kb = base + lane;
-      const bool on = kb <= qt && flags[kb] != 0u;
+      const bool on = kb <= last && flags[kb] != 0u;
       const uint32_t m = __ballot_sync(0xffffffffu, on);
       if (on) out[1 + count + __popc(m & ((1u << lane) - 1u))] = kb;
       count += __popc(m);
