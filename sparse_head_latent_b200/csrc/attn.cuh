@@ -78,6 +78,30 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// (x0, x1) <- (x0 * c + b, x1 * c + b): one packed f32x2 FMA (one issue
+// slot for two elements).
+__device__ __forceinline__ void fma2_scalar(float& x0, float& x1, float c, float b) {
+  asm("{\n\t.reg .b64 t, u, v;\n\t"
+      "mov.b64 t, {%0, %1};\n\t"
+      "mov.b64 u, {%2, %2};\n\t"
+      "mov.b64 v, {%3, %3};\n\t"
+      "fma.rn.f32x2 t, t, u, v;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(c), "f"(b));
+}
+
+// (a0, a1) += (x0, x1): one packed f32x2 add.
+__device__ __forceinline__ void add2(float& a0, float& a1, float x0, float x1) {
+  asm("{\n\t.reg .b64 t, u;\n\t"
+      "mov.b64 t, {%0, %1};\n\t"
+      "mov.b64 u, {%2, %3};\n\t"
+      "add.f32x2 t, t, u;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -198,16 +222,21 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // thread, so "S_t(j+1) is ready" also means "PV_t(j) is done".
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, 0, 1);
-      const uint32_t sV = smem_u32(smem + AttnSmem::V);
+      // Shared-memory descriptors are built once; a K step only moves the
+      // start address (bits 0-13, in 16-byte units), which never carries.
+      const uint64_t dQ[2] = {smem_desc_sw128(smem_u32(smem + AttnSmem::QA), 16, 1024),
+                              smem_desc_sw128(smem_u32(smem + AttnSmem::QB), 16, 1024)};
+      const uint64_t dK[2] = {smem_desc_sw128(smem_u32(smem + AttnSmem::K0), 16, 1024),
+                              smem_desc_sw128(smem_u32(smem + AttnSmem::K1), 16, 1024)};
+      const uint64_t dV = smem_desc_sw128(smem_u32(smem + AttnSmem::V), 16384, 1024);
       int issued = 0;
       auto qk = [&](int t, int j) {
-        const uint32_t sK = smem_u32(smem + ((j & 1) ? AttnSmem::K1 : AttnSmem::K0));
-        const uint32_t sQ = smem_u32(smem + (t ? AttnSmem::QB : AttnSmem::QA));
+        const uint64_t q0 = t ? dQ[1] : dQ[0];
+        const uint64_t k0 = (j & 1) ? dK[1] : dK[0];
 #pragma unroll
         for (int k = 0; k < 12; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          umma_ss(tmem + tmem_s(t), smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024),
-                  idesc_qk, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+          umma_ss(tmem + tmem_s(t), q0 + off, k0 + off, idesc_qk, k > 0 ? 1u : 0u);
         }
         umma_commit(bar(kBarSFull0 + t));
         ++issued;
@@ -215,7 +244,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       auto pv = [&](int t, int j) {
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + tmem_o(t), tmem + tmem_s(t) + k * 8, smem_desc_sw128(sV + k * 2048, 16384, 1024), idesc_pv,
+          umma_ts(tmem + tmem_o(t), tmem + tmem_s(t) + k * 8, dV + ((k * 2048) >> 4), idesc_pv,
                   (j > 0 || k > 0) ? 1u : 0u);
         ++issued;
       };
@@ -290,15 +319,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           for (int i = 0; i < 64; ++i) pk[i] = 0u;
         } else {
           float x[128];
-          {
-            uint32_t a0[32], a1[32];
-            tmem_ld32x2(tS, tS + 32, a0, a1);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) { x[i] = __uint_as_float(a0[i]); x[32 + i] = __uint_as_float(a1[i]); }
-            tmem_ld32x2(tS + 64, tS + 96, a0, a1);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) { x[64 + i] = __uint_as_float(a0[i]); x[96 + i] = __uint_as_float(a1[i]); }
-          }
+          tmem_ld128(tS, *reinterpret_cast<uint32_t(*)[128]>(x));
           // Selection: unselected scores become -inf (raw domain; the scale is
           // positive, so the max commutes with it).
           const bool all_sel = (bw[0] & bw[1] & bw[2] & bw[3]) == 0xffffffffu;
@@ -334,12 +355,14 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           float sm[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) sm[i] = 0.f;
+          // The argument and the row sums use packed f32x2 FMA/add (one issue
+          // slot per two elements); the softmax is bound by issue slots.
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            const float p0 = ex2_approx(fmaf(x[2 * i], c, nb));
-            const float p1 = ex2_approx(fmaf(x[2 * i + 1], c, nb));
-            sm[(2 * i) & 7] += p0;
-            sm[(2 * i + 1) & 7] += p1;
+            fma2_scalar(x[2 * i], x[2 * i + 1], c, nb);
+            const float p0 = ex2_approx(x[2 * i]);
+            const float p1 = ex2_approx(x[2 * i + 1]);
+            add2(sm[2 * (i & 3)], sm[2 * (i & 3) + 1], p0, p1);
             pk[i] = pack_f16x2(p0, p1);
           }
           l_run = l_run * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
@@ -357,12 +380,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           }
         }
         // P (f16 pairs) over the first half of S_t.
-        {
-          uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-          tmem_st32(tS, p0);
-          tmem_st32(tS + 32, p1);
-        }
+        tmem_st64(tS, pk);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kBarPFull0 + t));
