@@ -129,11 +129,12 @@ bool map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t i
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 tensor [B, T, inner] (row pitch inner*2 bytes), box [1, 128, 64].
-bool map_3d_bt(CUtensorMap* m, const void* base, uint64_t inner, uint64_t T, uint64_t B) {
+// bf16 tensor [B, T, inner] (row pitch inner*2 bytes), box [1, box_rows, 64];
+// rows past T read as zero.
+bool map_3d_bt(CUtensorMap* m, const void* base, uint64_t inner, uint64_t T, uint64_t B, uint32_t box_rows = 128) {
   const cuuint64_t dims[3] = {inner, T, B};
   const cuuint64_t strides[2] = {inner * 2, inner * 2 * T};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t es[3] = {1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -224,7 +225,7 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
     if (entry == MLA_ENTRY_PREFILL) w.attn = take(rows * H * kDv * 2);
     if (has_topk) {
       w.bitmap = take(static_cast<size_t>(d.B) * (nq * (nq + 1) / 2) * 128 * 16);
-      w.blocks = take(static_cast<size_t>(d.B) * nq * (nq + 1) * 4);
+      w.blocks = take(static_cast<size_t>(d.B) * ((nq + 3) / 4) * (nq + 2) * 4);
     }
   }
   if (fp8 && (attend || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
@@ -309,7 +310,7 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
         topk, d.B, d.T, d.topk, nq, static_cast<uint4*>(bitmap));
   });
   if (rc != MLA_OK) return rc;
-  dim3 grid((nq + 1) / 2, d.B);
+  dim3 grid((nq + 3) / 4, d.B);
   return timed_launch(0, st, [&] {
     mla::topk_block_list_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4*>(bitmap), nq,
                                                       static_cast<int32_t*>(blocks));
@@ -318,17 +319,19 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
 
 int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, const void* kvh, const void* k_pe,
                      const void* bitmap, const void* blocks, float scale, void* attn, cudaStream_t st) {
-  CUtensorMap tq, tkv, tpe;
+  // Q tiles and V blocks are 128 rows; each CTA of a pair loads 64 keys of K.
+  CUtensorMap tq, tk, tv, tpe;
+  const uint64_t kv_inner = static_cast<uint64_t>(d.H) * (kDn + kDv);
   if (!map_3d_bt(&tq, q, static_cast<uint64_t>(d.H) * (kDn + kDr), d.T, d.B) ||
-      !map_3d_bt(&tkv, kvh, static_cast<uint64_t>(d.H) * (kDn + kDv), d.T, d.B) ||
-      !map_3d_bt(&tpe, k_pe, kDr, d.T, d.B))
+      !map_3d_bt(&tk, kvh, kv_inner, d.T, d.B, 64) || !map_3d_bt(&tv, kvh, kv_inner, d.T, d.B) ||
+      !map_3d_bt(&tpe, k_pe, kDr, d.T, d.B, 64))
     return MLA_ERR_CUDA;
   mla::AttnParams p;
   p.B = d.B;
   p.T = d.T;
   p.H = d.H;
   p.nq = (d.T + 127) / 128;
-  p.npairs = (p.nq + 1) / 2;
+  p.ngroups = (p.nq + 3) / 4;
   // Heads per scheduling group: the largest of 8, 4, 2, 1 that divides H and
   // keeps the group's K/V (T x 512 bytes per head and batch) near 48 MB or less.
   p.hgroup = 1;
@@ -343,10 +346,22 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.blocks = static_cast<const int32_t*>(blocks);
   p.attn = static_cast<__nv_bfloat16*>(attn);
   p.err = ds->err;
-  const int64_t grid = static_cast<int64_t>(d.B) * p.npairs * d.H;
-  return timed_launch(3, st, [&] {
-    mla::sparse_mla_attn_kernel<<<static_cast<unsigned>(grid), mla::kAttnThreads, mla::AttnSmem::BYTES, st>>>(tq, tkv, tpe, p);
-  });
+  const int64_t pairs = static_cast<int64_t>(d.B) * p.ngroups * d.H;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(mla::kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = mla::AttnSmem::BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+  const int rc = timed_launch(3, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::sparse_mla_attn_kernel, tq, tk, tv, tpe, p); });
+  return le != cudaSuccess ? MLA_ERR_CUDA : rc;
 }
 
 }  // namespace

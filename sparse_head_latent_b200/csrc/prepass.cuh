@@ -9,19 +9,20 @@
 //
 // Layout (per batch b, 128-query tile qt, 128-key block kb <= qt):
 //   bitmap[b][qt*(qt+1)/2 + kb][row 0..127][4 x u32]   (bit c of the 128 = key kb*128 + c)
-//   blocks[b][pair][0] = number of key blocks with any bit set for either
-//   query tile of the pair (tiles 2*pair and 2*pair+1, which the attention
-//   kernel processes together), blocks[b][pair][1 + i] = their indices,
-//   ascending.
+//   blocks[b][g][0] = number of key blocks with any bit set for a query
+//   tile of group g (tiles 4g .. 4g+3, which one CTA pair of the attention
+//   kernel processes together), blocks[b][g][1] = how many of those lie at
+//   or below tile 4g+1 (the blocks the group's first two tiles can see),
+//   blocks[b][g][2 + i] = the indices, ascending. Row pitch nq + 2.
 //
 // Two launches:
 //   topk_bitmap_rows_kernel   one warp per query row (B * tiles * 128 rows):
 //                             shared-memory atomics build the row's bits,
 //                             then the row's words are written for every
 //                             causal block (rows past T get zeros)
-//   topk_block_list_kernel    one CTA per (tile pair, batch): OR of each
-//                             block's bits over both tiles, ballot-compacted
-//                             into the pair's list
+//   topk_block_list_kernel    one CTA per (tile group, batch): OR of each
+//                             block's bits over the group's tiles,
+//                             ballot-compacted into the group's list
 // No global atomics; the result is deterministic.
 #pragma once
 
@@ -67,13 +68,14 @@ topk_bitmap_rows_kernel(const int32_t* __restrict__ topk_idx, int B, int T, int 
 __global__ void __launch_bounds__(128)
 topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __restrict__ blocks) {
   __shared__ uint32_t flags[MLA_MAX_T / 128];
-  const int pair = blockIdx.x, b = blockIdx.y;
-  const int qa = 2 * pair, qb = 2 * pair + 1;
-  const int last = qb < nq ? qb : qa;  // highest key block either tile can see
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int q0 = 4 * g;
+  const int last = min(q0 + 3, nq - 1);     // highest key block a tile of the group can see
+  const int last_a = min(q0 + 1, nq - 1);   // highest one of the group's first two tiles
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int kb = warp; kb <= last; kb += 4) {
     uint32_t acc = 0;
-    for (int qt = qa; qt <= last; ++qt) {
+    for (int qt = q0; qt <= last; ++qt) {
       if (kb > qt) continue;  // outside this tile's causal triangle
       const uint4* blk = bitmap + (b * tri_index(nq, 0) + tri_index(qt, kb)) * 128;
 #pragma unroll
@@ -87,16 +89,22 @@ topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __rest
   }
   __syncthreads();
   if (warp == 0) {
-    int32_t* out = blocks + (static_cast<int64_t>(b) * nq + pair) * (nq + 1);
-    int count = 0;
+    const int ngroups = (nq + 3) / 4;
+    int32_t* out = blocks + (static_cast<int64_t>(b) * ngroups + g) * (nq + 2);
+    int count = 0, count_a = 0;
     for (int base = 0; base <= last; base += 32) {
       const int kb = base + lane;
       const bool on = kb <= last && flags[kb] != 0u;
       const uint32_t m = __ballot_sync(0xffffffffu, on);
-      if (on) out[1 + count + __popc(m & ((1u << lane) - 1u))] = kb;
+      const uint32_t ma = __ballot_sync(0xffffffffu, on && kb <= last_a);
+      if (on) out[2 + count + __popc(m & ((1u << lane) - 1u))] = kb;
       count += __popc(m);
+      count_a += __popc(ma);
     }
-    if (lane == 0) out[0] = count;
+    if (lane == 0) {
+      out[0] = count;
+      out[1] = count_a;
+    }
   }
 }
 

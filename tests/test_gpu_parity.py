@@ -82,6 +82,12 @@ ATTEND_CASES = {
     "short_rows": dict(B=1, T=77, H=2, topk=100),
     "four_tiles": dict(B=1, T=512, H=2, topk=96),
     "fp8_sparse": dict(B=2, T=200, H=2, topk=24, fp8=True),
+    # Several groups of four query tiles; the last group is ragged: six tiles
+    # (no second super-tile), nine tiles (a lone tile whose pair partner lies
+    # past T).
+    "groups_ragged_sparse": dict(B=2, T=700, H=2, topk=200),
+    "groups_lone_tile_causal": dict(B=1, T=1100, H=2, topk=None),
+    "groups_lone_tile_sparse": dict(B=1, T=1100, H=3, topk=300),
 }
 
 
