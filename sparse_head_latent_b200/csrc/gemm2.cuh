@@ -238,7 +238,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(acce0 + 8 * a, 0));
+      if (lane == 0) mbar_arrive_remote(mapa_shared(acce0 + 8 * a, 0));
     }
     if (lane == 0) bulk_wait_group<0>();
   }
