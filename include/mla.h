@@ -63,11 +63,20 @@ typedef enum {
                               "Down projection" page: fmt e4m3, weight_block_size [128, 128]) */
 } mla_wdtype;
 
+/* How the attention rows are computed (same result up to rounding; see
+ * mla_attend). AUTO picks per group of 512 query rows by a cost model. */
+typedef enum {
+  MLA_PATH_AUTO = 0,
+  MLA_PATH_BLOCK_DENSE = 1,  /* every row: up-projected keys, 128-key blocks */
+  MLA_PATH_ABSORBED = 2      /* every row with a topk_idx: absorbed form over the gathered keys */
+} mla_path;
+
 typedef struct {
   int B, T, H;
   int d_nope, d_rope, d_v, d_latent, d_model;
   int topk;          /* entries per row of topk_idx (ignored when topk_idx == NULL) */
   mla_wdtype wdtype; /* storage of W_kvb and W_o */
+  mla_path path;     /* MLA_PATH_AUTO (0) unless a caller forces one path */
 } mla_dims;
 
 /* Entry points, for mla_workspace_bytes(). */
@@ -108,7 +117,20 @@ int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_
  *   scale    : softmax scale applied to q.k, finite and > 0 (192^-0.5 for
  *              these models)
  *   attn_out : bf16 [B, T, H, 128]. A query with no surviving key gets 0.
- * Softmax in fp32 (exp2 form); P and V enter the PV product as bf16. */
+ * Softmax in fp32 (exp2 form); P and V enter the PV product as bf16 (f16).
+ * Two ways to the same result (dims->path):
+ *   block-dense: up-project every key (k_nope_h, v_h = W_kvb rows applied to
+ *     kv_latent), then per (query tile, 128-key block holding a selected key)
+ *     scores, mask, softmax, value mix;
+ *   absorbed (DeepSeek-V2 "Multi-Head Latent Attention", the decode form
+ *     applied to prefill rows): per query row, q_nope of each head is
+ *     multiplied into W_kvb's k_nope rows (q_abs, 512 wide), scored against
+ *     the row's selected latent rows [kv_latent | k_pe] only, the softmax
+ *     weights mix the latent rows, and W_kvb's v rows map the 512-wide
+ *     result to the head's 128 values. It costs 2176 instead of 640 FLOP
+ *     per (head, key) but visits only the selected keys, so it wins for rows
+ *     whose causal prefix is several times longer than topk.
+ * The absorbed path needs topk_idx; without it every row is block-dense. */
 int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent,
                const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
                const int32_t* topk_idx, float scale, void* attn_out,
@@ -176,9 +198,11 @@ int mla_device_status(mla_stream_t stream, int* device_error);
  * the calls above on this host thread's library instance; mla_profile_end()
  * synchronises those events and writes, per kernel class, the total
  * milliseconds and launch count, then stops recording.
- * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention,
- * 4 W_o GEMM. Arrays must hold MLA_PROFILE_CLASSES entries. */
-#define MLA_PROFILE_CLASSES 5
+ * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention
+ * (block-dense), 4 W_o GEMM, 5 per-row key lists, 6 absorb and un-absorb
+ * GEMMs, 7 attention (absorbed). Arrays must hold MLA_PROFILE_CLASSES
+ * entries. */
+#define MLA_PROFILE_CLASSES 8
 int mla_profile_begin(void);
 int mla_profile_end(float* ms_total, int* launches);
 

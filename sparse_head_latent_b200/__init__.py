@@ -2,7 +2,8 @@
 
 The C ABI (include/mla.h, libmla_b200.so) runs the whole block in CUDA
 kernels: W_kvb up-projection (tcgen05 GEMM), top-k selection bitmap,
-fused sparse-causal attention, W_o output projection (tcgen05 GEMM).
+fused sparse-causal attention (block-dense, or absorbed over each row's
+gathered latent keys for long rows), W_o output projection (tcgen05 GEMM).
 This package is its thin ctypes binding; the library is loaded on first
 use and a missing build is an error, never a fallback.
 """
@@ -11,6 +12,9 @@ from .mla import (  # noqa: F401
     MLA_ENTRY_KV_UPPROJECT,
     MLA_ENTRY_OUT_PROJECT,
     MLA_ENTRY_PREFILL,
+    MLA_PATH_ABSORBED,
+    MLA_PATH_AUTO,
+    MLA_PATH_BLOCK_DENSE,
     MlaDims,
     MlaError,
     PrefillPipeline,

@@ -48,7 +48,8 @@ namespace mla {
 
 struct AttnParams {
   int B, T, H, nq;
-  int ngroups;                  // ceil(nq / 4) groups of four query tiles
+  int ngroups;                  // groups of four query tiles to run: groups 0 .. ngroups-1
+  int gpitch;                   // ceil(nq / 4): groups per batch element in `blocks`
   int hgroup;                   // heads per scheduling group (divides H)
   float scale_log2;             // softmax scale * log2(e)
   const uint4* bitmap;          // selection bitmap, NULL = causal mask only
@@ -94,42 +95,6 @@ enum : int {
   kBarDrain = 16    // leader: drain after an abort
 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// (x0, x1) <- (x0 * c + b, x1 * c + b): one packed f32x2 FMA (one issue
-// slot for two elements).
-__device__ __forceinline__ void fma2_scalar(float& x0, float& x1, float c, float b) {
-  asm("{\n\t.reg .b64 t, u, v;\n\t"
-      "mov.b64 t, {%0, %1};\n\t"
-      "mov.b64 u, {%2, %2};\n\t"
-      "mov.b64 v, {%3, %3};\n\t"
-      "fma.rn.f32x2 t, t, u, v;\n\t"
-      "mov.b64 {%0, %1}, t;\n\t}"
-      : "+f"(x0), "+f"(x1)
-      : "f"(c), "f"(b));
-}
-
-// (a0, a1) += (x0, x1): one packed f32x2 add.
-__device__ __forceinline__ void add2(float& a0, float& a1, float x0, float x1) {
-  asm("{\n\t.reg .b64 t, u;\n\t"
-      "mov.b64 t, {%0, %1};\n\t"
-      "mov.b64 u, {%2, %3};\n\t"
-      "add.f32x2 t, t, u;\n\t"
-      "mov.b64 {%0, %1}, t;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(x0), "f"(x1));
-}
-
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKpe,
@@ -167,7 +132,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   // if its first tile does and visits the blocks of the list up to its last
   // existing tile: a prefix of the list, which is ascending.
   const bool has_b = q0 + 2 < p.nq;
-  const int32_t* blist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.ngroups + grp) * (p.nq + 2) : nullptr;
+  const int32_t* blist = p.blocks ? p.blocks + (static_cast<int64_t>(b) * p.gpitch + grp) * (p.nq + 2) : nullptr;
   int nA, nB;
   if (blist) {
     nA = blist[1];

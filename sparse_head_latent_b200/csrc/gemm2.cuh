@@ -27,12 +27,14 @@ namespace mla {
 // V_F16: the output columns [128, 256) of every 256-column tile are stored
 // as f16 instead of bf16. With N = H*256 that is the v half of each head of
 // the up-projection, which the attention kernel consumes as f16.
-template <bool B_MN_MAJOR_, bool V_F16_ = false>
+// BN_: output tile width per pair, 256 or 128.
+template <bool B_MN_MAJOR_, bool V_F16_ = false, int BN_ = 256>
 struct Gemm2Cfg {
+  static_assert(BN_ == 256 || BN_ == 128, "tile width");
   static constexpr int BM = 256;       // per CTA pair
-  static constexpr int BN = 256;       // per CTA pair
+  static constexpr int BN = BN_;       // per CTA pair
   static constexpr int HM = 128;       // A rows per CTA
-  static constexpr int HN = 128;       // B columns per CTA
+  static constexpr int HN = BN_ / 2;   // B columns per CTA
   static constexpr int BK = 64;
   static constexpr bool B_MN_MAJOR = B_MN_MAJOR_;
   static constexpr bool V_F16 = V_F16_;
@@ -50,6 +52,18 @@ struct Gemm2Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
+// A batch of independent GEMMs with the same M, N, K that differ only in
+// where their operands sit in the three tensor maps: GEMM i reads A at
+// column a_col0 + i * a_col_step, B at row b_row0 + i * b_row_step (rows are
+// N for a K-major B, K for an N-major B) and writes C at column
+// c_col0 + i * c_col_step. One plain GEMM is {1, 0, 0, 0, 0, 0, 0}.
+struct GemmBatch {
+  int count;
+  int a_col0, a_col_step;
+  int b_row0, b_row_step;
+  int c_col0, c_col_step;
+};
+
 // Spin for about `ns` nanoseconds (used only to let in-flight copies land on
 // the abort path, where this CTA cannot observe the leader's barrier).
 __device__ __forceinline__ void spin_ns(uint64_t ns) {
@@ -61,7 +75,7 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, int* err) {
+                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, const GemmBatch bt, int* err) {
   constexpr int BK = Cfg::BK, S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -109,7 +123,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
   const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
   const int num_n = N / Cfg::BN;
-  const int num_tiles = num_m * num_n;
+  const int num_tiles = num_m * num_n * bt.count;
   const int num_kb = K / BK;
   const int pair = static_cast<int>(blockIdx.x) >> 1;
   const int num_pairs = static_cast<int>(gridDim.x) >> 1;
@@ -120,9 +134,11 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int it = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % num_m, nt = tile / num_m;
+        const int mt = tile % num_m, nt = (tile / num_m) % num_n, bi = tile / (num_m * num_n);
         const int arow = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM;
         const int bcol = nt * Cfg::BN + static_cast<int>(rank) * Cfg::HN;
+        const int acol0 = bt.a_col0 + bi * bt.a_col_step;
+        const int brow0 = bt.b_row0 + bi * bt.b_row_step;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -134,12 +150,13 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * Cfg::STAGE_BYTES);
           const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t sb = sa + Cfg::A_BYTES;
-          tma_load_2d_pair(sa, &tmA, full_leader, kb * BK, arow);
+          tma_load_2d_pair(sa, &tmA, full_leader, acol0 + kb * BK, arow);
           if constexpr (!Cfg::B_MN_MAJOR) {
-            tma_load_2d_pair(sb, &tmB, full_leader, kb * BK, bcol);
+            tma_load_2d_pair(sb, &tmB, full_leader, kb * BK, brow0 + bcol);
           } else {
-            tma_load_2d_pair(sb, &tmB, full_leader, bcol, kb * BK);
-            tma_load_2d_pair(sb + BK * 128, &tmB, full_leader, bcol + 64, kb * BK);
+#pragma unroll
+            for (int h = 0; h < Cfg::HN / 64; ++h)
+              tma_load_2d_pair(sb + h * BK * 128, &tmB, full_leader, bcol + 64 * h, brow0 + kb * BK);
           }
         }
       }
@@ -193,15 +210,21 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* bufs = epi + (warp - 2) * 2 * Cfg::EPI_BUF;
     int t = 0, nbuf = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
-      const int mt = tile % num_m, nt = tile / num_m;
+      const int mt = tile % num_m, nt = (tile / num_m) % num_n, bi = tile / (num_m * num_n);
       const int a = t & 1;
       const uint32_t aph = (t >> 1) & 1;
       if (!warp_wait(accf0 + 8 * a, aph, ab, kErrWaitMma)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * 256;
       const int row0 = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM + q * 32;
+      // A warp whose 32 rows all lie past M has nothing to store. It must
+      // then skip the staging too: the two staging buffers alternate per
+      // issued store, and `wait_group.read 1` before a buffer is rewritten
+      // only covers the store two issues back if every staged chunk was
+      // stored (otherwise the previous tile's last store could still be
+      // reading the buffer being overwritten).
 #pragma unroll 1
-      for (int c = 0; c < Cfg::BN / 64; ++c) {
+      for (int c = 0; c < Cfg::BN / 64 && row0 < M; ++c) {
         uint32_t r0[32], r1[32];
         tmem_ld32x2(tb + c * 64, tb + c * 64 + 32, r0, r1);
         uint8_t* buf = bufs + (nbuf & 1) * Cfg::EPI_BUF;
@@ -230,8 +253,8 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && row0 < M) {
-          tma_store_2d(&tmC, smem_u32(buf), nt * Cfg::BN + c * 64, row0);
+        if (lane == 0) {
+          tma_store_2d(&tmC, smem_u32(buf), bt.c_col0 + bi * bt.c_col_step + nt * Cfg::BN + c * 64, row0);
           bulk_commit_group();
         }
         ++nbuf;

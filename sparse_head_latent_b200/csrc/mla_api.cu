@@ -14,6 +14,7 @@
 
 #include "../../include/mla.h"
 #include "attn.cuh"
+#include "attn_abs.cuh"
 #include "dequant.cuh"
 #include "gemm2.cuh"
 #include "prepass.cuh"
@@ -27,7 +28,8 @@ namespace {
 constexpr int kDn = 128, kDr = 64, kDv = 128, kL = 512, kD = 7168;
 using Gemm2Kvb = mla::Gemm2Cfg<false>;  // latent x W_kvb^T  (B stored [N, K])
 using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as f16 for the attention
-using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N])
+using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
+using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
 
 // ------------------------------------------------------------------ device state
 
@@ -37,6 +39,7 @@ struct DeviceState {
   int sms = 0;
   int pairs_kvb = 0;   // CTA pairs of the pair GEMMs that fit on the device at once
   int pairs_wo = 0;
+  int pairs_unabs = 0;
   int* err = nullptr;  // address of g_mla_device_error on this device
 };
 
@@ -91,11 +94,16 @@ int device_state(DeviceState** out) {
                                       Gemm2Wo::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2KvbAttn>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2KvbAttn::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2Unabs>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Unabs::SMEM_BYTES) == cudaSuccess;
       if (ok) {
         st.pairs_kvb = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, Gemm2Kvb::SMEM_BYTES);
         st.pairs_wo = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, Gemm2Wo::SMEM_BYTES);
-        ok = st.pairs_kvb > 0 && st.pairs_wo > 0;
+        st.pairs_unabs = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Unabs>, Gemm2Unabs::SMEM_BYTES);
+        ok = st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_unabs > 0;
       }
+      ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      mla::AbsSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AttnSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::topk_bitmap_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -194,8 +202,36 @@ constexpr int64_t kMaxRows = int64_t(1) << 24;  // B*T limit (int32 tile coordin
 
 struct WsLayout {
   size_t kvh = kNone, attn = kNone, bitmap = kNone, blocks = kNone, wkvb = kNone, wo = kNone;
+  size_t qabs = kNone, olat = kNone, lists = kNone, counts = kNone;  // absorbed path, one chunk of rows
+  int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
+  int abs_chunk = 0;   // absorbed rows processed per pass
+  int kpad = 0;        // pitch of the per-row key lists
   size_t total = 0;
 };
+
+// Absorbed rows are processed in passes of at most this many rows of one
+// batch element, which bounds the workspace (q_abs and o_lat are
+// rows x H x 1 KB each).
+constexpr int kAbsChunkRows = 2048;
+// Cost model for MLA_PATH_AUTO: a tile group goes absorbed when its middle
+// row's causal prefix exceeds this many times the selection size. Per
+// (head, key) the absorbed form does 2176 FLOP against 640 for the
+// block-dense form, which visits the whole prefix, and runs at a lower
+// fraction of the tensor-core peak.
+constexpr int kAbsorbRatio = 5;
+
+// First tile group that runs on the absorbed path (== number of groups when
+// none does).
+int absorbed_first_group(const mla_dims& d, bool has_topk) {
+  const int nq = (d.T + 127) / 128;
+  const int ng = (nq + 3) / 4;
+  if (!has_topk || d.path == MLA_PATH_BLOCK_DENSE) return ng;
+  if (d.path == MLA_PATH_ABSORBED) return 0;
+  const int64_t k = d.topk < d.T ? d.topk : d.T;
+  for (int g = 0; g < ng; ++g)
+    if (int64_t(512) * g + 256 > int64_t(kAbsorbRatio) * k) return g;
+  return ng;
+}
 
 int check_dims(const mla_dims* d) {
   if (d == nullptr) return MLA_ERR_NULL;
@@ -204,6 +240,8 @@ int check_dims(const mla_dims* d) {
   if (d->wdtype != MLA_W_BF16 && d->wdtype != MLA_W_E4M3_BLOCK128) return MLA_ERR_UNSUPPORTED;
   if (d->B < 0 || d->T < 0 || d->H < 1 || d->T > MLA_MAX_T) return MLA_ERR_SHAPE;
   if (static_cast<int64_t>(d->B) * d->T > kMaxRows) return MLA_ERR_SHAPE;
+  if (d->path != MLA_PATH_AUTO && d->path != MLA_PATH_BLOCK_DENSE && d->path != MLA_PATH_ABSORBED)
+    return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -221,11 +259,23 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
   const bool fp8 = d.wdtype == MLA_W_E4M3_BLOCK128;
   const bool attend = entry == MLA_ENTRY_ATTEND || entry == MLA_ENTRY_PREFILL;
   if (attend) {
-    w.kvh = take(rows * H * (kDn + kDv) * 2);
+    w.g_abs = absorbed_first_group(d, has_topk);
+    if (w.g_abs > 0) w.kvh = take(rows * H * (kDn + kDv) * 2);  // block-dense rows only
     if (entry == MLA_ENTRY_PREFILL) w.attn = take(rows * H * kDv * 2);
     if (has_topk) {
       w.bitmap = take(static_cast<size_t>(d.B) * (nq * (nq + 1) / 2) * 128 * 16);
       w.blocks = take(static_cast<size_t>(d.B) * ((nq + 3) / 4) * (nq + 2) * 4);
+    }
+    const int64_t abs_rows = int64_t(d.T) - int64_t(512) * w.g_abs;
+    if (abs_rows > 0 && d.B > 0) {
+      w.abs_chunk = static_cast<int>(abs_rows < kAbsChunkRows ? abs_rows : kAbsChunkRows);
+      const int k = d.topk < d.T ? d.topk : d.T;
+      w.kpad = (k + 63) / 64 * 64;
+      const size_t ch = static_cast<size_t>(w.abs_chunk);
+      w.qabs = take(ch * H * kL * 2);
+      w.olat = take(ch * H * kL * 2);
+      w.lists = take(ch * static_cast<size_t>(w.kpad) * 4);
+      w.counts = take(ch * 4);
     }
   }
   if (fp8 && (attend || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
@@ -251,10 +301,12 @@ int launch_dequant(const DeviceState* ds, const void* codes, const float* scale,
   });
 }
 
+constexpr mla::GemmBatch kOneGemm = {1, 0, 0, 0, 0, 0, 0};
+
 template <class Cfg>
 int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M,
-                     int N, int K, int* err, int cls, cudaStream_t st) {
-  const int tiles = ((M + Cfg::BM - 1) / Cfg::BM) * (N / Cfg::BN);
+                     int N, int K, int* err, int cls, cudaStream_t st, const mla::GemmBatch& bt = kOneGemm) {
+  const int tiles = ((M + Cfg::BM - 1) / Cfg::BM) * (N / Cfg::BN) * bt.count;
   const int pairs = tiles < pairs_max ? tiles : pairs_max;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -270,7 +322,7 @@ int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb
   cfg.numAttrs = 1;
   cudaError_t le = cudaSuccess;
   const int rc = timed_launch(
-      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, err); });
+      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, bt, err); });
   return le != cudaSuccess ? MLA_ERR_CUDA : rc;
 }
 
@@ -317,8 +369,10 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
   });
 }
 
+// Block-dense attention for tile groups [0, ngroups_run).
 int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, const void* kvh, const void* k_pe,
-                     const void* bitmap, const void* blocks, float scale, void* attn, cudaStream_t st) {
+                     const void* bitmap, const void* blocks, float scale, void* attn, int ngroups_run,
+                     cudaStream_t st) {
   // Q tiles and V blocks are 128 rows; each CTA of a pair loads 64 keys of K.
   CUtensorMap tq, tk, tv, tpe;
   const uint64_t kv_inner = static_cast<uint64_t>(d.H) * (kDn + kDv);
@@ -331,7 +385,8 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.T = d.T;
   p.H = d.H;
   p.nq = (d.T + 127) / 128;
-  p.ngroups = (p.nq + 3) / 4;
+  p.gpitch = (p.nq + 3) / 4;
+  p.ngroups = ngroups_run;
   // Heads per scheduling group: the largest of 8, 4, 2, 1 that divides H and
   // keeps the group's K/V (T x 512 bytes per head and batch) near 48 MB or less.
   p.hgroup = 1;
@@ -362,6 +417,75 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   cudaError_t le = cudaSuccess;
   const int rc = timed_launch(3, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::sparse_mla_attn_kernel, tq, tk, tv, tpe, p); });
   return le != cudaSuccess ? MLA_ERR_CUDA : rc;
+}
+
+// Selected keys of rows s0 .. s0+rows-1 of batch element b, from the bitmap.
+int launch_row_lists(const mla_dims& d, const void* bitmap, int b, int s0, int rows, int kpad, int32_t* lists,
+                     int32_t* counts, cudaStream_t st) {
+  const int nq = (d.T + 127) / 128;
+  const unsigned grid = static_cast<unsigned>((rows + mla::kPrepassWarps - 1) / mla::kPrepassWarps);
+  return timed_launch(5, st, [&] {
+    mla::topk_row_lists_kernel<<<grid, 32 * mla::kPrepassWarps, 0, st>>>(static_cast<const uint4*>(bitmap), nq, d.T,
+                                                                          b, s0, rows, kpad, lists, counts);
+  });
+}
+
+// q_abs[r, h, :] = q[r, h, 0:128] . W_kvb[h*256 + (0..127), :] for `rows`
+// consecutive rows: one GEMM per head (M = rows, N = 512, K = 128).
+int launch_gemm_absorb(const DeviceState* ds, int H, int rows, const void* q_rows, const void* wk, void* qabs,
+                       cudaStream_t st) {
+  CUtensorMap ta, tb, tc;
+  const uint64_t qw = static_cast<uint64_t>(H) * (kDn + kDr);
+  if (!map_2d(&ta, q_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qw, rows, qw * 2, 64, 128) ||
+      !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64, 64) ||
+      !map_2d(&tc, qabs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
+              static_cast<uint64_t>(H) * kL * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const mla::GemmBatch bt = {H, 0, kDn + kDr, 0, kDn + kDv, 0, kL};
+  return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, rows, kL, kDn, ds->err, 6, st, bt);
+}
+
+// attn[r, h, :] = o_lat[r, h, :] . W_kvb[h*256 + 128 + (0..127), :]^T: one
+// GEMM per head (M = rows, N = 128, K = 512).
+int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* olat, const void* wk, void* attn_rows,
+                         cudaStream_t st) {
+  CUtensorMap ta, tb, tc;
+  if (!map_2d(&ta, olat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
+              static_cast<uint64_t>(H) * kL * 2, 64, 128) ||
+      !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64,
+              Gemm2Unabs::HN) ||
+      !map_2d(&tc, attn_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kDv, rows,
+              static_cast<uint64_t>(H) * kDv * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const mla::GemmBatch bt = {H, 0, kL, kDn, kDn + kDv, 0, kDv};
+  return launch_gemm_pair<Gemm2Unabs>(ds->pairs_unabs, ta, tb, tc, rows, kDv, kL, ds->err, 6, st, bt);
+}
+
+// Absorbed attention for `rows` rows (one CTA per row and group of 64 heads).
+int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const void* lat, const void* k_pe, int rows,
+                              int key_row0, int kpad, const int32_t* lists, const int32_t* counts, const void* qabs,
+                              const void* q_rows, void* olat, float scale, cudaStream_t st) {
+  CUtensorMap tl, tp;
+  const uint64_t all = static_cast<uint64_t>(d.B) * d.T;
+  if (!map_2d(&tl, lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, all, kL * 2, 64, 1) ||
+      !map_2d(&tp, k_pe, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDr, all, kDr * 2, 64, 1))
+    return MLA_ERR_CUDA;
+  mla::AbsParams p;
+  p.rows = rows;
+  p.H = d.H;
+  p.kpad = kpad;
+  p.key_row0 = key_row0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lists = lists;
+  p.counts = counts;
+  p.qabs = static_cast<const __nv_bfloat16*>(qabs);
+  p.q = static_cast<const __nv_bfloat16*>(q_rows);
+  p.olat = static_cast<__nv_bfloat16*>(olat);
+  p.err = ds->err;
+  return timed_launch(7, st, [&] {
+    mla::absorbed_attn_kernel<<<static_cast<unsigned>(rows * ((d.H + 63) / 64)), mla::kAbsThreads, mla::AbsSmem::BYTES,
+                                 st>>>(tl, tp, p);
+  });
 }
 
 }  // namespace
@@ -397,9 +521,22 @@ int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay,
 int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* q,
                const void* lat, const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
                const int32_t* topk_idx, float scale, void* attn, cudaStream_t st) {
-  void* kvh = ws_at(ws, lay.kvh);
-  int rc = run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, /*v_f16=*/true, st);
-  if (rc != MLA_OK) return rc;
+  const int nq = (d.T + 127) / 128;
+  const int ng = (nq + 3) / 4;
+  const void* wk = W_kvb;
+  int rc = MLA_OK;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    void* dq = ws_at(ws, lay.wkvb);
+    rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st);
+    if (rc != MLA_OK) return rc;
+    wk = dq;
+  }
+  void* kvh = nullptr;
+  if (lay.g_abs > 0) {  // up-projected keys, for the block-dense rows only
+    kvh = ws_at(ws, lay.kvh);
+    rc = launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, /*v_f16=*/true, st);
+    if (rc != MLA_OK) return rc;
+  }
   void* bitmap = nullptr;
   void* blocks = nullptr;
   if (topk_idx != nullptr) {
@@ -408,7 +545,32 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
     rc = launch_prepass(ds, d, topk_idx, bitmap, blocks, st);
     if (rc != MLA_OK) return rc;
   }
-  return launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, st);
+  if (lay.g_abs > 0) {
+    rc = launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, lay.g_abs, st);
+    if (rc != MLA_OK) return rc;
+  }
+  if (lay.g_abs >= ng) return MLA_OK;
+  // Absorbed rows [512 * g_abs, T) of every batch element, in passes.
+  void* qabs = ws_at(ws, lay.qabs);
+  void* olat = ws_at(ws, lay.olat);
+  int32_t* lists = reinterpret_cast<int32_t*>(ws_at(ws, lay.lists));
+  int32_t* counts = reinterpret_cast<int32_t*>(ws_at(ws, lay.counts));
+  const size_t qrow = static_cast<size_t>(d.H) * (kDn + kDr) * 2, arow = static_cast<size_t>(d.H) * kDv * 2;
+  for (int b = 0; b < d.B; ++b) {
+    for (int s0 = 512 * lay.g_abs; s0 < d.T; s0 += lay.abs_chunk) {
+      const int rows = d.T - s0 < lay.abs_chunk ? d.T - s0 : lay.abs_chunk;
+      const size_t r0 = static_cast<size_t>(b) * d.T + s0;
+      const void* q_rows = static_cast<const uint8_t*>(q) + r0 * qrow;
+      void* attn_rows = static_cast<uint8_t*>(attn) + r0 * arow;
+      if ((rc = launch_row_lists(d, bitmap, b, s0, rows, lay.kpad, lists, counts, st)) != MLA_OK) return rc;
+      if ((rc = launch_gemm_absorb(ds, d.H, rows, q_rows, wk, qabs, st)) != MLA_OK) return rc;
+      if ((rc = launch_attention_absorbed(ds, d, lat, k_pe, rows, b * d.T, lay.kpad, lists, counts, qabs, q_rows,
+                                          olat, scale, st)) != MLA_OK)
+        return rc;
+      if ((rc = launch_gemm_unabsorb(ds, d.H, rows, olat, wk, attn_rows, st)) != MLA_OK) return rc;
+    }
+  }
+  return MLA_OK;
 }
 
 int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* attn,

@@ -108,4 +108,55 @@ topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __rest
   }
 }
 
+// Selected keys of query rows, ascending, for the absorbed path: row i of
+// the launch is query s = s0 + i of batch b (s < T). One warp per row reads
+// the row's bitmap words block by block, counts the set bits per 128-key
+// block, scans the counts across the warp and writes each block's keys at
+// its offset. lists[i][0 .. count) are the keys, padded with key 0 up to the
+// next multiple of 64 (the gather loads whole 64-key blocks; the padding is
+// masked by the count). Row pitch kpad >= count, a multiple of 64.
+__global__ void __launch_bounds__(32 * kPrepassWarps)
+topk_row_lists_kernel(const uint4* __restrict__ bitmap, int nq, int T, int b, int s0, int rows, int kpad,
+                      int32_t* __restrict__ lists, int32_t* __restrict__ counts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = static_cast<int>(blockIdx.x) * kPrepassWarps + warp;
+  if (i >= rows) return;
+  const int s = s0 + i;
+  int32_t* out = lists + static_cast<int64_t>(i) * kpad;
+  int count = 0;
+  if (s < T) {
+    const int qt = s >> 7, r = s & 127;
+    const uint4* row = bitmap + (static_cast<int64_t>(b) * tri_index(nq, 0) + tri_index(qt, 0)) * 128 + r;
+    for (int base = 0; base <= qt; base += 32) {
+      const int kb = base + lane;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (kb <= qt) w = __ldg(row + static_cast<int64_t>(kb) * 128);
+      const int c = __popc(w.x) + __popc(w.y) + __popc(w.z) + __popc(w.w);
+      int incl = c;  // inclusive scan of the per-block counts
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      int pos = count + incl - c;
+      const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t m = words[q];
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          m &= m - 1;
+          if (pos < kpad) out[pos] = kb * 128 + q * 32 + bit;
+          ++pos;
+        }
+      }
+      count += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  if (count > kpad) count = kpad;
+  const int padded = (count + 63) & ~63;
+  for (int j = count + lane; j < padded; j += 32) out[j] = 0;
+  if (lane == 0) counts[i] = count;
+}
+
 }  // namespace mla

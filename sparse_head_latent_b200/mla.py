@@ -20,8 +20,10 @@ _lib = None
 
 MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL = 0, 1, 2, 3
 MLA_W_BF16, MLA_W_E4M3_BLOCK128 = 0, 1
-MLA_PROFILE_CLASSES = 5
-PROFILE_CLASS_NAMES = ("topk_prepass", "weight_dequant", "gemm_kvb", "attention", "gemm_wo")
+MLA_PROFILE_CLASSES = 8
+MLA_PATH_AUTO, MLA_PATH_BLOCK_DENSE, MLA_PATH_ABSORBED = 0, 1, 2
+PROFILE_CLASS_NAMES = ("topk_prepass", "weight_dequant", "gemm_kvb", "attention", "gemm_wo", "row_lists",
+                       "gemm_absorb", "attention_absorbed")
 D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL = 128, 64, 128, 512, 7168
 
 
@@ -29,7 +31,7 @@ class MlaDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
                 ("d_nope", ctypes.c_int), ("d_rope", ctypes.c_int), ("d_v", ctypes.c_int),
                 ("d_latent", ctypes.c_int), ("d_model", ctypes.c_int),
-                ("topk", ctypes.c_int), ("wdtype", ctypes.c_int)]
+                ("topk", ctypes.c_int), ("wdtype", ctypes.c_int), ("path", ctypes.c_int)]
 
 
 class MlaError(RuntimeError):
@@ -102,9 +104,9 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_dims(B, T, H, topk=0, fp8=False) -> MlaDims:
+def make_dims(B, T, H, topk=0, fp8=False, path=MLA_PATH_AUTO) -> MlaDims:
     return MlaDims(int(B), int(T), int(H), D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL, int(topk),
-                   MLA_W_E4M3_BLOCK128 if fp8 else MLA_W_BF16)
+                   MLA_W_E4M3_BLOCK128 if fp8 else MLA_W_BF16, int(path))
 
 
 def _wtype(w: torch.Tensor) -> bool:
@@ -142,11 +144,11 @@ def mla_kv_upproject(kv_latent, W_kvb, W_kvb_scale=None, kvh_out=None, workspace
 
 
 def mla_attend(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale=192 ** -0.5,
-               attn_out=None, workspace=None, stream=None):
+               attn_out=None, workspace=None, stream=None, path=MLA_PATH_AUTO):
     """q [B,T,H,192], kv_latent [B,T,512], k_pe [B,T,64] (bf16) -> attn bf16 [B,T,H,128]."""
     B, T, H, _ = q.shape
     topk = 0 if topk_idx is None else topk_idx.shape[-1]
-    dims = make_dims(B, T, H, topk, _wtype(W_kvb))
+    dims = make_dims(B, T, H, topk, _wtype(W_kvb), path)
     if topk_idx is not None and topk_idx.dtype != torch.int32:
         raise ValueError("topk_idx must be int32")
     if attn_out is None:
@@ -195,7 +197,7 @@ def mla_out_project(attn, W_o, W_o_scale=None, out=None, workspace=None, stream=
 
 
 def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk_idx=None,
-                scale=192 ** -0.5, out=None, workspace=None, stream=None):
+                scale=192 ** -0.5, out=None, workspace=None, stream=None, path=MLA_PATH_AUTO):
     """The whole attend block: -> out bf16 [B, T, 7168]."""
     B, T, H, _ = q.shape
     topk = 0 if topk_idx is None else topk_idx.shape[-1]
@@ -204,7 +206,7 @@ def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None
         raise ValueError("W_kvb and W_o must use the same storage type")
     if topk_idx is not None and topk_idx.dtype != torch.int32:
         raise ValueError("topk_idx must be int32")
-    dims = make_dims(B, T, H, topk, fp8)
+    dims = make_dims(B, T, H, topk, fp8, path)
     if out is None:
         out = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=q.device)
     ws, nbytes = _workspace(dims, MLA_ENTRY_PREFILL, topk_idx is not None, workspace, q.device)

@@ -48,7 +48,7 @@ def _dims(**kw):
 
 
 def test_workspace_sizes(lib):
-    d = _dims()
+    d = _dims(path=mla.MLA_PATH_BLOCK_DENSE)
     kvh = 256 * 4 * 256 * 2
     assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_KV_UPPROJECT, False) == 0
     assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_OUT_PROJECT, False) == 0
@@ -64,6 +64,23 @@ def test_workspace_sizes(lib):
     assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_OUT_PROJECT, False) == 4 * 128 * 7168 * 2
     assert mla.mla_workspace_bytes(_dims(d_model=4096), mla.MLA_ENTRY_ATTEND, False) == 0
     assert mla.mla_workspace_bytes(d, 9, False) == 0
+
+
+def test_workspace_sizes_absorbed_path(lib):
+    # Absorbed rows need no up-projected keys but q_abs and o_lat (rows x H x
+    # 512 bf16 each) and the per-row key lists (k rounded up to 64, int32).
+    T, H, k = 256, 4, 16
+    d = _dims(path=mla.MLA_PATH_ABSORBED)
+    nq = 2
+    bitmap = nq * (nq + 1) // 2 * 128 * 16
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    want = up(bitmap) + up((nq + 3) // 4 * (nq + 2) * 4) + 2 * up(T * H * 512 * 2) + up(T * 64 * 4) + up(T * 4)
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, True) == want
+    # without top-k indices every row is block-dense whatever the request
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, False) == T * H * 256 * 2
+    # the automatic choice sends this shape (k = 16, rows up to 256) to the absorbed path
+    assert mla.mla_workspace_bytes(_dims(), mla.MLA_ENTRY_ATTEND, True) == want
+    assert mla.mla_workspace_bytes(_dims(path=3), mla.MLA_ENTRY_ATTEND, True) == 0
 
 
 def _attend(lib, d, ptrs=None, scale=0.07, ws=None, nbytes=0):
