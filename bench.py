@@ -40,7 +40,7 @@ import synth  # noqa: E402
 METRIC = "sparse MLA prefill TFLOP/s and queries/s (T=4096,H=128,top-k 2048); % of bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "attn.cuh", "prepass.cuh", "dequant.cuh", "mla_api.cu")
+KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "attn.cuh", "attn_abs.cuh", "prepass.cuh", "dequant.cuh", "mla_api.cu")
 
 
 def parse_args(argv=None):

@@ -15,7 +15,9 @@
 //
 // Work item: one CTA per (query row, group of 64 heads): M = 64 heads
 // against the row's selected keys, gathered in blocks of 64 from the latent
-// rows by TMA (tile::gather4, four arbitrary rows per instruction). The list
+// rows by three warps of 16-byte cp.async copies (coalesced along each key's
+// row, written into the 128-byte-swizzled operand layout; a TMA gather4
+// moved only ~8 bytes per clock per SM for these 128-byte rows). The list
 // of selected keys comes from the causal selection bitmap (ascending,
 // duplicates and out-of-range entries already gone).
 //
@@ -32,10 +34,10 @@
 //   PV:   M=64, N=256 (twice), K=64, A = P, B = the key stage's latent chunks
 //         read N-major (the same bytes: a key's 64 latent values per row)
 //
-// CTA = 192 threads: warp 0 gathers, warp 1 allocates tensor memory and
-// issues the UMMAs, warps 2..5 run the softmax (lanes 16..31 own the heads'
-// S rows; lanes 0..15 own the same heads' O rows, for the rescale and the
-// epilogue).
+// CTA = 256 threads: warps 0, 6, 7 gather, warp 1 allocates tensor memory
+// and issues the UMMAs, warps 2..5 run the softmax (lanes 16..31 own the
+// heads' S rows; lanes 0..15 own the same heads' O rows, for the rescale and
+// the epilogue).
 #pragma once
 
 #include "ptx.cuh"
@@ -52,6 +54,8 @@ struct AbsParams {
   const int32_t* counts;       // [rows]
   const __nv_bfloat16* qabs;   // [rows][H][512]
   const __nv_bfloat16* q;      // [rows][H][192] (rope at 128..191)
+  const __nv_bfloat16* lat;    // kv_latent [B*T][512]
+  const __nv_bfloat16* kpe;    // k_pe [B*T][64]
   __nv_bfloat16* olat;         // [rows][H][512]
   int* err;
 };
@@ -67,12 +71,14 @@ struct AbsSmem {
 };
 static_assert(AbsSmem::BYTES <= 232448, "shared memory per CTA");
 
-constexpr int kAbsThreads = 192;
+constexpr int kAbsThreads = 256;
+constexpr int kAbsLoaders = 96;              // threads of the three gather warps
 constexpr uint32_t kAbsLaneHi = 16u << 16;   // lane offset of Q and S
+constexpr int kL_abs = 512;                  // latent width
 constexpr uint32_t kAbsColS = 288;           // first S column (after Q's 288)
 
 enum : int {
-  kAbsKFull0 = 0,    // per stage: the gathered keys landed
+  kAbsKFull0 = 0,    // per stage: the gathered keys landed (every gather thread)
   kAbsKEmpty0 = 3,   // per stage: the UMMAs reading it are done
   kAbsQReady = 6,    // Q is in tensor memory (four softmax warps)
   kAbsSFull0 = 7,    // per S buffer
@@ -83,8 +89,7 @@ enum : int {
 };
 
 __global__ void __launch_bounds__(kAbsThreads, 1)
-absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_constant__ CUtensorMap tmPe,
-                     const AbsParams p) {
+absorbed_attn_kernel(const AbsParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AbsSmem::BARS);
@@ -108,7 +113,7 @@ absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_con
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < AbsSmem::K_STAGES; ++i) {
-      mbar_init(bar(kAbsKFull0 + i), 1);
+      mbar_init(bar(kAbsKFull0 + i), kAbsLoaders);
       mbar_init(bar(kAbsKEmpty0 + i), 1);
     }
     mbar_init(bar(kAbsQReady), 4);
@@ -121,10 +126,6 @@ absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_con
     *abort_word = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmLat);
-    prefetch_tmap(&tmPe);
-  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
@@ -135,34 +136,44 @@ absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_con
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_word, p.err};
 
-  if (warp == 0) {
-    if (lane == 0 && n > 0) {
+  if (warp == 0 || warp >= 6) {
+    if (n > 0) {
       // ---------------- gather: block j = keys [64j, 64j + 64) of the row's
-      // list into stage j % 3, four rows per instruction, nine column chunks
-      int issued = 0;
+      // list into stage j % 3 as nine [64 keys x 64] chunks (eight latent,
+      // one rope). Loader warp w (0..2) takes keys w, w + 3, ...; the lanes
+      // copy a key's 72 16-byte pieces (1152 bytes: 1024 latent + 128 rope)
+      // in three coalesced instructions. The block's 64 indices are read
+      // once per warp (two per lane) and broadcast by shuffle. Each thread
+      // waits for its own copies, makes them visible to the tensor core's
+      // (async) proxy, and arrives on the stage's barrier.
+      const int w = warp == 0 ? 0 : warp - 5;
+      const uint8_t* lat = reinterpret_cast<const uint8_t*>(p.lat);
+      const uint8_t* pe = reinterpret_cast<const uint8_t*>(p.kpe);
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
         const int s = j % AbsSmem::K_STAGES;
-        if (!(ok = mbar_wait(bar(kAbsKEmpty0 + s), ((j / AbsSmem::K_STAGES) & 1) ^ 1, ab, kErrWaitMma))) break;
-        const uint32_t fb = bar(kAbsKFull0 + s);
-        mbar_arrive_expect_tx(fb, AbsSmem::K_STAGE);
-        const uint32_t dst = smem_u32(smem + s * AbsSmem::K_STAGE);
-        const int4* kq = reinterpret_cast<const int4*>(keys + 64 * j);
-#pragma unroll 1
-        for (int g = 0; g < 16; ++g) {
-          const int4 k4 = __ldg(kq + g);
-          const int r0 = p.key_row0 + k4.x, r1 = p.key_row0 + k4.y;
-          const int r2 = p.key_row0 + k4.z, r3 = p.key_row0 + k4.w;
+        if (!(ok = warp_wait(bar(kAbsKEmpty0 + s), ((j / AbsSmem::K_STAGES) & 1) ^ 1, ab, kErrWaitMma))) break;
+        const uint32_t stage = smem_u32(smem + s * AbsSmem::K_STAGE);
+        const int2 kk = __ldg(reinterpret_cast<const int2*>(keys + 64 * j) + lane);  // keys 2l, 2l+1
+#pragma unroll 2
+        for (int i = w; i < 64; i += 3) {
+          const int kx = __shfl_sync(0xffffffffu, kk.x, i >> 1);
+          const int ky = __shfl_sync(0xffffffffu, kk.y, i >> 1);
+          const int64_t krow = static_cast<int64_t>(p.key_row0) + ((i & 1) ? ky : kx);
+          const uint32_t drow = stage + i * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            tma_gather4_2d(dst + c * AbsSmem::CHUNK + g * 512, &tmLat, fb, 64 * c, r0, r1, r2, r3);
-          tma_gather4_2d(dst + 8 * AbsSmem::CHUNK + g * 512, &tmPe, fb, 0, r0, r1, r2, r3);
+          for (int r = 0; r < 3; ++r) {
+            const int pc = static_cast<int>(lane) + 32 * r;  // piece of this key: chunk pc / 8, column pc % 8
+            if (pc < 72) {
+              const int c = pc >> 3, e = pc & 7;
+              const uint8_t* src = c < 8 ? lat + krow * (kL_abs * 2) + pc * 16 : pe + krow * 128 + e * 16;
+              cp_async16(drow + c * AbsSmem::CHUNK + ((e ^ (i & 7)) << 4), src);
+            }
+          }
         }
-        ++issued;
-      }
-      if (!ok) {
-        for (int i = (issued > AbsSmem::K_STAGES ? issued - AbsSmem::K_STAGES : 0); i < issued; ++i)
-          mbar_wait_drain(bar(kAbsKFull0 + i % AbsSmem::K_STAGES), (i / AbsSmem::K_STAGES) & 1);
+        cp_async_commit_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar(kAbsKFull0 + s));
       }
     }
   } else if (warp == 1) {
@@ -220,7 +231,7 @@ absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_con
       }
     }
   } else {
-    // ---------------- softmax warps. Warp w covers the tensor-memory lanes of
+    // ---------------- softmax warps (2..5). Warp w covers the tensor-memory lanes of
     // sub-partition q = w % 4: lanes 16..31 of it hold the S rows (and Q) of
     // heads 16q .. 16q+15 of this half, lanes 0..15 the O rows of the same
     // heads, so a lane and the lane 16 above it work on the same head.
@@ -238,24 +249,31 @@ absorbed_attn_kernel(const __grid_constant__ CUtensorMap tmLat, const __grid_con
       // 0..15 store zeros into O's columns, which PV(0) overwrites.
       const __nv_bfloat16* qa = p.qabs + (static_cast<int64_t>(row) * p.H + hp) * 512;
       const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(row) * p.H + hp) * 192 + 128;
+      // Software-pipelined: the loads of chunk cc + 1 are in flight while
+      // chunk cc is stored (a load-then-store round trip per chunk would put
+      // nine global-load latencies on every CTA's path to its first UMMA).
+      const bool qload = srow && hvalid;
+      auto load_chunk = [&](int cc, uint4 (&w)[8]) {
+        const uint4* src = reinterpret_cast<const uint4*>(cc < 8 ? qa + 64 * cc : qr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = qload ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      };
+      uint4 cur[8], nxt[8];
+      load_chunk(0, cur);
 #pragma unroll 1
       for (int cc = 0; cc < 9; ++cc) {
+        if (cc + 1 < 9) load_chunk(cc + 1, nxt);
         uint32_t v[32];
-        if (srow && hvalid) {
-          const uint4* src = reinterpret_cast<const uint4*>(cc < 8 ? qa + 64 * cc : qr);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 w = __ldg(src + i);
-            v[4 * i] = w.x;
-            v[4 * i + 1] = w.y;
-            v[4 * i + 2] = w.z;
-            v[4 * i + 3] = w.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        for (int i = 0; i < 8; ++i) {
+          v[4 * i] = cur[i].x;
+          v[4 * i + 1] = cur[i].y;
+          v[4 * i + 2] = cur[i].z;
+          v[4 * i + 3] = cur[i].w;
         }
         tmem_st32(tq + 32u * cc, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
       tc_fence_before();
       __syncwarp();

@@ -214,11 +214,12 @@ struct WsLayout {
 // rows x H x 1 KB each).
 constexpr int kAbsChunkRows = 2048;
 // Cost model for MLA_PATH_AUTO: a tile group goes absorbed when its middle
-// row's causal prefix exceeds this many times the selection size. Per
-// (head, key) the absorbed form does 2176 FLOP against 640 for the
-// block-dense form, which visits the whole prefix, and runs at a lower
-// fraction of the tensor-core peak.
-constexpr int kAbsorbRatio = 5;
+// row's causal prefix exceeds this many times the selection size. Measured
+// on B200 at T = 32768, H = 128, top-k 2048: the block-dense kernel costs
+// about 80 ps per (row, prefix key) for all heads, the absorbed kernel about
+// 870 ps per (row, selected key) (2176 instead of 640 FLOP per head and key,
+// M = 64 UMMAs, and every 64-head group gathers the row's keys from L2).
+constexpr int kAbsorbRatio = 11;
 
 // First tile group that runs on the absorbed path (== number of groups when
 // none does).
@@ -465,11 +466,6 @@ int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* ola
 int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const void* lat, const void* k_pe, int rows,
                               int key_row0, int kpad, const int32_t* lists, const int32_t* counts, const void* qabs,
                               const void* q_rows, void* olat, float scale, cudaStream_t st) {
-  CUtensorMap tl, tp;
-  const uint64_t all = static_cast<uint64_t>(d.B) * d.T;
-  if (!map_2d(&tl, lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, all, kL * 2, 64, 1) ||
-      !map_2d(&tp, k_pe, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kDr, all, kDr * 2, 64, 1))
-    return MLA_ERR_CUDA;
   mla::AbsParams p;
   p.rows = rows;
   p.H = d.H;
@@ -480,11 +476,13 @@ int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const vo
   p.counts = counts;
   p.qabs = static_cast<const __nv_bfloat16*>(qabs);
   p.q = static_cast<const __nv_bfloat16*>(q_rows);
+  p.lat = static_cast<const __nv_bfloat16*>(lat);
+  p.kpe = static_cast<const __nv_bfloat16*>(k_pe);
   p.olat = static_cast<__nv_bfloat16*>(olat);
   p.err = ds->err;
   return timed_launch(7, st, [&] {
     mla::absorbed_attn_kernel<<<static_cast<unsigned>(rows * ((d.H + 63) / 64)), mla::kAbsThreads, mla::AbsSmem::BYTES,
-                                 st>>>(tl, tp, p);
+                                 st>>>(p);
   });
 }
 
