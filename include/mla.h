@@ -84,6 +84,7 @@ typedef struct {
 #define MLA_ENTRY_ATTEND 1
 #define MLA_ENTRY_OUT_PROJECT 2
 #define MLA_ENTRY_PREFILL 3
+#define MLA_ENTRY_DECODE 4
 
 /* Device workspace bytes that `entry` needs for these dims (has_topk = 1
  * if a topk_idx will be passed). 0 when nothing is needed or the dims are
@@ -155,6 +156,32 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent,
                 float scale, void* out, void* workspace, size_t ws_bytes,
                 mla_stream_t stream);
 
+/* Decode: one new position per sequence against its cache (DeepSeek-V3.2-
+ * Exp "Sparse attention" at generation time, where the pages score the
+ * cached latent directly: the absorbed form of DeepSeek-V2 "Multi-Head
+ * Latent Attention"). Equals row s = T-1 of mla_prefill for a sequence whose
+ * first T-1 positions are the cache, up to rounding.
+ *   dims     : B sequences, T = cache length including the new position
+ *              (the query sits at s = T-1), H, topk, wdtype; path ignored
+ *   q        : bf16 [B, H, 192] of the new position (nope then rope)
+ *   kv_latent: bf16 [B, T, 512] latent cache, the new position's row last
+ *   k_pe     : bf16 [B, T, 64] rotated rope keys of the cache
+ *   W_kvb, W_kvb_scale, W_o, W_o_scale: as for mla_prefill
+ *   topk_idx : int32 [B, topk] selected cache positions of the new query,
+ *              any order; duplicates select once, entries outside [0, T)
+ *              select nothing. NULL = every position.
+ *   out      : bf16 [B, 7168]. A sequence with no selected key gets 0 before
+ *              W_o (so 0).
+ * Steps: per-sequence key lists, q_abs = q_nope . W_UK per head (tcgen05
+ * GEMM), attention over the gathered latent keys (the absorbed kernel),
+ * attn = W_UV . o_lat per head, then W_o. Workspace: mla_workspace_bytes(
+ * dims, MLA_ENTRY_DECODE, topk_idx != NULL). Errors as for mla_prefill. */
+int mla_decode(const mla_dims* dims, const void* q, const void* kv_latent,
+               const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
+               const void* W_o, const float* W_o_scale, const int32_t* topk_idx,
+               float scale, void* out, void* workspace, size_t ws_bytes,
+               mla_stream_t stream);
+
 /* mla_attend without a caller-supplied workspace (no counterpart on the
  * pages: it exists for callers that cannot hand the library device memory).
  *
@@ -199,8 +226,8 @@ int mla_device_status(mla_stream_t stream, int* device_error);
  * synchronises those events and writes, per kernel class, the total
  * milliseconds and launch count, then stops recording.
  * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention
- * (block-dense), 4 W_o GEMM, 5 per-row key lists, 6 absorb and un-absorb
- * GEMMs, 7 attention (absorbed). Arrays must hold MLA_PROFILE_CLASSES
+ * (block-dense), 4 W_o GEMM, 5 per-row key lists (prefill and decode),
+ * 6 absorb and un-absorb GEMMs, 7 attention (absorbed). Arrays must hold MLA_PROFILE_CLASSES
  * entries. */
 #define MLA_PROFILE_CLASSES 8
 int mla_profile_begin(void);

@@ -9,6 +9,7 @@ use and a missing build is an error, never a fallback.
 """
 from .mla import (  # noqa: F401
     MLA_ENTRY_ATTEND,
+    MLA_ENTRY_DECODE,
     MLA_ENTRY_KV_UPPROJECT,
     MLA_ENTRY_OUT_PROJECT,
     MLA_ENTRY_PREFILL,
@@ -23,6 +24,7 @@ from .mla import (  # noqa: F401
     make_dims,
     mla_attend,
     mla_attend_static,
+    mla_decode,
     mla_device_status,
     mla_kv_upproject,
     mla_out_project,

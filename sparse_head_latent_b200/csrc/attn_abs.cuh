@@ -45,10 +45,13 @@
 namespace mla {
 
 struct AbsParams {
-  int rows;                    // query rows of this launch (consecutive s of one batch element)
+  int rows;                    // query rows of this launch
   int H;
   int kpad;                    // pitch of `lists`
-  int key_row0;                // row of key t = 0 of this batch element in the latent tensors (b * T)
+  // Row of key t = 0 for query row r in the latent tensors: key_row0 +
+  // (r / rows_per_seq) * seq_stride (prefill: the launch's rows share one
+  // sequence; decode: one row per sequence, seq_stride = T).
+  int key_row0, rows_per_seq, seq_stride;
   float scale_log2;            // softmax scale * log2(e)
   const int32_t* lists;        // [rows][kpad] selected keys, ascending, padded with 0
   const int32_t* counts;       // [rows]
@@ -110,6 +113,7 @@ absorbed_attn_kernel(const AbsParams p) {
   const int count = p.counts[row];
   const int n = (count + 63) >> 6;                      // 64-key blocks
   const int32_t* keys = p.lists + static_cast<int64_t>(row) * p.kpad;
+  const int key_base = p.key_row0 + (row / p.rows_per_seq) * p.seq_stride;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < AbsSmem::K_STAGES; ++i) {
@@ -159,7 +163,7 @@ absorbed_attn_kernel(const AbsParams p) {
         for (int i = w; i < 64; i += 3) {
           const int kx = __shfl_sync(0xffffffffu, kk.x, i >> 1);
           const int ky = __shfl_sync(0xffffffffu, kk.y, i >> 1);
-          const int64_t krow = static_cast<int64_t>(p.key_row0) + ((i & 1) ? ky : kx);
+          const int64_t krow = static_cast<int64_t>(key_base) + ((i & 1) ? ky : kx);
           const uint32_t drow = stage + i * 128;
 #pragma unroll
           for (int r = 0; r < 3; ++r) {

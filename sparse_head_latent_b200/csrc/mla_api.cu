@@ -279,8 +279,19 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
       w.counts = take(ch * 4);
     }
   }
-  if (fp8 && (attend || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
-  if (fp8 && (entry == MLA_ENTRY_PREFILL || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+  if (entry == MLA_ENTRY_DECODE && d.B > 0) {
+    const size_t B = d.B;
+    const int k = has_topk ? (d.topk < d.T ? d.topk : d.T) : d.T;
+    w.kpad = (k + 63) / 64 * 64;
+    w.qabs = take(B * H * kL * 2);
+    w.olat = take(B * H * kL * 2);
+    w.lists = take(B * static_cast<size_t>(w.kpad) * 4);
+    w.counts = take(B * 4);
+    w.attn = take(B * H * kDv * 2);
+  }
+  const bool dec = entry == MLA_ENTRY_DECODE;
+  if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
+  if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
   w.total = off;
   return w;
 }
@@ -431,6 +442,15 @@ int launch_row_lists(const mla_dims& d, const void* bitmap, int b, int s0, int r
   });
 }
 
+// Decode: selected cache positions of each sequence's new query.
+int launch_decode_lists(const mla_dims& d, const int32_t* topk, int kpad, int32_t* lists, int32_t* counts,
+                        cudaStream_t st) {
+  return timed_launch(5, st, [&] {
+    mla::decode_row_lists_kernel<<<static_cast<unsigned>(d.B), mla::kDecodeListThreads, 0, st>>>(
+        topk, d.T, topk ? d.topk : 0, kpad, lists, counts);
+  });
+}
+
 // q_abs[r, h, :] = q[r, h, 0:128] . W_kvb[h*256 + (0..127), :] for `rows`
 // consecutive rows: one GEMM per head (M = rows, N = 512, K = 128).
 int launch_gemm_absorb(const DeviceState* ds, int H, int rows, const void* q_rows, const void* wk, void* qabs,
@@ -464,13 +484,16 @@ int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* ola
 
 // Absorbed attention for `rows` rows (one CTA per row and group of 64 heads).
 int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const void* lat, const void* k_pe, int rows,
-                              int key_row0, int kpad, const int32_t* lists, const int32_t* counts, const void* qabs,
+                              int key_row0, int rows_per_seq, int seq_stride, int kpad, const int32_t* lists,
+                              const int32_t* counts, const void* qabs,
                               const void* q_rows, void* olat, float scale, cudaStream_t st) {
   mla::AbsParams p;
   p.rows = rows;
   p.H = d.H;
   p.kpad = kpad;
   p.key_row0 = key_row0;
+  p.rows_per_seq = rows_per_seq;
+  p.seq_stride = seq_stride;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.lists = lists;
   p.counts = counts;
@@ -562,8 +585,8 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
       void* attn_rows = static_cast<uint8_t*>(attn) + r0 * arow;
       if ((rc = launch_row_lists(d, bitmap, b, s0, rows, lay.kpad, lists, counts, st)) != MLA_OK) return rc;
       if ((rc = launch_gemm_absorb(ds, d.H, rows, q_rows, wk, qabs, st)) != MLA_OK) return rc;
-      if ((rc = launch_attention_absorbed(ds, d, lat, k_pe, rows, b * d.T, lay.kpad, lists, counts, qabs, q_rows,
-                                          olat, scale, st)) != MLA_OK)
+      if ((rc = launch_attention_absorbed(ds, d, lat, k_pe, rows, b * d.T, rows, 0, lay.kpad, lists, counts, qabs,
+                                          q_rows, olat, scale, st)) != MLA_OK)
         return rc;
       if ((rc = launch_gemm_unabsorb(ds, d.H, rows, olat, wk, attn_rows, st)) != MLA_OK) return rc;
     }
@@ -583,6 +606,38 @@ int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& la
   return launch_gemm_wo(ds, d.B * d.T, d.H, attn, wo, out, st);
 }
 
+// Decode: one new query per sequence (row s = T-1) against the cache, in the
+// absorbed form.
+int run_decode(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* q,
+               const void* lat, const void* k_pe, const void* W_kvb, const float* W_kvb_scale, const void* W_o,
+               const float* W_o_scale, const int32_t* topk_idx, float scale, void* out, cudaStream_t st) {
+  const void* wk = W_kvb;
+  int rc = MLA_OK;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    void* dq = ws_at(ws, lay.wkvb);
+    if ((rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st)) != MLA_OK) return rc;
+    wk = dq;
+  }
+  void* qabs = ws_at(ws, lay.qabs);
+  void* olat = ws_at(ws, lay.olat);
+  void* attn = ws_at(ws, lay.attn);
+  int32_t* lists = reinterpret_cast<int32_t*>(ws_at(ws, lay.lists));
+  int32_t* counts = reinterpret_cast<int32_t*>(ws_at(ws, lay.counts));
+  if ((rc = launch_decode_lists(d, topk_idx, lay.kpad, lists, counts, st)) != MLA_OK) return rc;
+  if ((rc = launch_gemm_absorb(ds, d.H, d.B, q, wk, qabs, st)) != MLA_OK) return rc;
+  if ((rc = launch_attention_absorbed(ds, d, lat, k_pe, d.B, 0, 1, d.T, lay.kpad, lists, counts, qabs, q, olat, scale,
+                                      st)) != MLA_OK)
+    return rc;
+  if ((rc = launch_gemm_unabsorb(ds, d.H, d.B, olat, wk, attn, st)) != MLA_OK) return rc;
+  const void* wo = W_o;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    void* dq = ws_at(ws, lay.wo);
+    if ((rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st)) != MLA_OK) return rc;
+    wo = dq;
+  }
+  return launch_gemm_wo(ds, d.B, d.H, attn, wo, out, st);
+}
+
 bool fp8_scales_ok(const mla_dims* d, const float* s) { return d->wdtype != MLA_W_E4M3_BLOCK128 || s != nullptr; }
 
 }  // namespace
@@ -590,7 +645,7 @@ bool fp8_scales_ok(const mla_dims* d, const float* s) { return d->wdtype != MLA_
 extern "C" {
 
 size_t mla_workspace_bytes(const mla_dims* dims, int entry, int has_topk) {
-  if (check_dims(dims) != MLA_OK || entry < MLA_ENTRY_KV_UPPROJECT || entry > MLA_ENTRY_PREFILL) return 0;
+  if (check_dims(dims) != MLA_OK || entry < MLA_ENTRY_KV_UPPROJECT || entry > MLA_ENTRY_DECODE) return 0;
   return ws_layout(*dims, entry, has_topk != 0).total;
 }
 
@@ -672,6 +727,28 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent, cons
   rc = run_attend(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, attn, st);
   if (rc != MLA_OK) return rc;
   return run_out_project(ds, *dims, lay, workspace, attn, W_o, W_o_scale, out, st);
+}
+
+int mla_decode(const mla_dims* dims, const void* q, const void* kv_latent, const void* k_pe, const void* W_kvb,
+               const float* W_kvb_scale, const void* W_o, const float* W_o_scale, const int32_t* topk_idx,
+               float scale, void* out, void* workspace, size_t ws_bytes, mla_stream_t stream) {
+  DeviceState* ds = nullptr;
+  WsLayout lay;
+  int rc = check_dims(dims);
+  if (rc != MLA_OK) return rc;
+  if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
+  if (!q || !kv_latent || !k_pe || !W_kvb || !W_o || !out || !fp8_scales_ok(dims, W_kvb_scale) ||
+      !fp8_scales_ok(dims, W_o_scale))
+    return MLA_ERR_NULL;
+  if (topk_idx != nullptr && dims->topk < 1) return MLA_ERR_SHAPE;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MLA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(W_o) ||
+      !aligned16(out) || !aligned16(W_kvb_scale) || !aligned16(W_o_scale) || !aligned16(topk_idx))
+    return MLA_ERR_ALIGN;
+  rc = begin_call(dims, MLA_ENTRY_DECODE, topk_idx != nullptr, workspace, ws_bytes, &ds, &lay);
+  if (rc != MLA_OK) return rc;
+  return run_decode(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, W_o, W_o_scale, topk_idx,
+                    scale, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* mla_status_str(int status) {

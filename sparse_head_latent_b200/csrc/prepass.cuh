@@ -159,4 +159,68 @@ topk_row_lists_kernel(const uint4* __restrict__ bitmap, int nq, int T, int b, in
   if (lane == 0) counts[i] = count;
 }
 
+// Decode: the selected cache positions of the one new query of sequence b
+// (topk_idx[b][0 .. k)), deduplicated and ascending, padded with 0 up to a
+// multiple of 64 (row pitch kpad); a NULL topk_idx selects every position
+// [0, T). One CTA per sequence sets the positions' bits in a T-bit set in
+// shared memory (entries outside [0, T) are dropped), then each thread
+// compacts a run of words at the offset a block-wide scan of the bit counts
+// gives it.
+constexpr int kDecodeListThreads = 256;
+
+__global__ void __launch_bounds__(kDecodeListThreads)
+decode_row_lists_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int kpad, int32_t* __restrict__ lists,
+                        int32_t* __restrict__ counts) {
+  __shared__ uint32_t bits[MLA_MAX_T / 32];
+  __shared__ int warp_total[kDecodeListThreads / 32];
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = (T + 31) / 32;
+  for (int w = tid; w < nw; w += kDecodeListThreads) {
+    uint32_t v = 0u;
+    if (topk_idx == nullptr) v = (w + 1) * 32 <= T ? 0xffffffffu : ((1u << (T - 32 * w)) - 1u);
+    bits[w] = v;
+  }
+  __syncthreads();
+  if (topk_idx != nullptr) {
+    const int32_t* idx = topk_idx + static_cast<int64_t>(b) * k;
+    for (int i = tid; i < k; i += kDecodeListThreads) {
+      const int32_t t = __ldg(idx + i);
+      if (t >= 0 && t < T) atomicOr(&bits[t >> 5], 1u << (t & 31));
+    }
+  }
+  __syncthreads();
+  const int wpt = (nw + kDecodeListThreads - 1) / kDecodeListThreads;  // words per thread
+  const int w0 = tid * wpt, w1 = min(w0 + wpt, nw);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(bits[w]);
+  int incl = c;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) warp_total[warp] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+  for (int i = 0; i < kDecodeListThreads / 32; ++i) {
+    if (i < warp) before += warp_total[i];
+    total += warp_total[i];
+  }
+  int32_t* out = lists + static_cast<int64_t>(b) * kpad;
+  int pos = before + incl - c;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t m = bits[w];
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1;
+      if (pos < kpad) out[pos] = w * 32 + bit;
+      ++pos;
+    }
+  }
+  const int count = total < kpad ? total : kpad;
+  const int padded = (count + 63) & ~63;
+  for (int j = count + tid; j < padded; j += kDecodeListThreads) out[j] = 0;
+  if (tid == 0) counts[b] = count;
+}
+
 }  // namespace mla

@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b20
 _lock = threading.Lock()
 _lib = None
 
-MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL = 0, 1, 2, 3
+MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL, MLA_ENTRY_DECODE = 0, 1, 2, 3, 4
 MLA_W_BF16, MLA_W_E4M3_BLOCK128 = 0, 1
 MLA_PROFILE_CLASSES = 8
 MLA_PATH_AUTO, MLA_PATH_BLOCK_DENSE, MLA_PATH_ABSORBED = 0, 1, 2
@@ -50,6 +50,8 @@ SIGNATURES = {
     "mla_out_project": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "mla_prefill": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                    ctypes.c_float, _VP, _VP, _SZ, _VP]),
+    "mla_decode": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                  ctypes.c_float, _VP, _VP, _SZ, _VP]),
     "mla_attend_static": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_float,
                                          _VP, _VP]),
     "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
@@ -214,6 +216,29 @@ def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None
     _check("mla_prefill", lib.mla_prefill(ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb),
                                           _ptr(W_kvb_scale), _ptr(W_o), _ptr(W_o_scale), _ptr(topk_idx),
                                           float(scale), _ptr(out), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def mla_decode(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk_idx=None,
+               scale=192 ** -0.5, out=None, workspace=None, stream=None):
+    """One new position per sequence against its cache: q [B,H,192], kv_latent [B,T,512], k_pe [B,T,64]
+    (the new position's cache row last), topk_idx int32 [B, topk] or None -> out bf16 [B, 7168]."""
+    B, H, _ = q.shape
+    T = kv_latent.shape[1]
+    topk = 0 if topk_idx is None else topk_idx.shape[-1]
+    fp8 = _wtype(W_kvb)
+    if _wtype(W_o) != fp8:
+        raise ValueError("W_kvb and W_o must use the same storage type")
+    if topk_idx is not None and topk_idx.dtype != torch.int32:
+        raise ValueError("topk_idx must be int32")
+    dims = make_dims(B, T, H, topk, fp8)
+    if out is None:
+        out = torch.empty(B, D_MODEL, dtype=torch.bfloat16, device=q.device)
+    ws, nbytes = _workspace(dims, MLA_ENTRY_DECODE, topk_idx is not None, workspace, q.device)
+    lib = load_library()
+    _check("mla_decode", lib.mla_decode(ctypes.byref(dims), _ptr(q), _ptr(kv_latent), _ptr(k_pe), _ptr(W_kvb),
+                                        _ptr(W_kvb_scale), _ptr(W_o), _ptr(W_o_scale), _ptr(topk_idx), float(scale),
+                                        _ptr(out), _ptr(ws), nbytes, _stream(stream)))
     return out
 
 
