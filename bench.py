@@ -50,6 +50,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--config", type=int, default=1)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--mode", choices=["prefill", "decode"], default="prefill",
+                   help="decode: one new position per sequence against a cache (B=64, T=32768 unless overridden)")
     p.add_argument("--e2e-steps", type=int, default=None, help="steps of the host-buffer run (default: --steps)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
@@ -409,6 +411,70 @@ def run_ours(args, rank, world, local):
 
 # ------------------------------------------------------------------ reference arm (CPU oracle)
 
+def run_decode(args, local):
+    """Decode throughput: B sequences, one new position each, against a cache
+    of T positions (the new one last), top-k selected positions per query.
+    Bound by HBM: the weights plus the gathered latent rows."""
+    import sparse_head_latent_b200 as mla
+
+    B, T = args.B or 64, args.T or 32768
+    H, k = args.H or 128, args.topk or 2048
+    x = synth.make_decode_inputs(B, T, H, k, seed=11)
+    dev = torch.device("cuda", local)
+    g = {n: v.to(dev) for n, v in x.tensors().items()}
+    dims = mla.make_dims(B, T, H, k, False)
+    ws = torch.empty(mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_DECODE, True), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, 7168, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mla.mla_decode(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], topk_idx=g["topk_idx"],
+                       scale=x.scale, out=out, workspace=ws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local).start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mla.mla_profile_begin()
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    prof = mla.mla_profile_end()
+    clocks.stop()
+    if mla.mla_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms = e0.elapsed_time(e1) / args.steps
+    sel = min(k, T)
+    compulsory = (H * 256 * 512 * 2 + H * 128 * 7168 * 2        # W_kvb, W_o
+                  + B * sel * (512 + 64) * 2                      # gathered latent and rope rows
+                  + B * H * 192 * 2 + B * k * 4 + B * 7168 * 2)  # q, top-k, out
+    flops = B * (2.0 * H * 128 * 512 * 2 + sel * H * 2 * (576 + 512) + 2.0 * H * 128 * 7168)
+    peaks, src = load_peaks()
+    gbs = compulsory / (ms * 1e-3) / 1e9
+    per = {n: {"launches": c, "avg_ms": round(t / max(c, 1), 5)} for n, (t, c) in prof.items() if c}
+    return {
+        "metric": "sparse MLA decode tokens/s (one new position per sequence, absorbed form)",
+        "value": round(B / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; no checkpoint)",
+        "config": {"workload": f"decode_B{B}_T{T}", "B": B, "T": T, "H": H, "topk": k, "weights": "bf16",
+                   "l2": "no flush: W_o alone (235 MB) exceeds the 126 MB L2"},
+        "algorithmic_gflop_per_step": round(flops / 1e9, 3),
+        "roofline": {"kernel": "whole decode step", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": f"{src} HBM copy bandwidth",
+                     "bytes_per_step": compulsory},
+        "per_kernel": per, "gpu_launches": sum(c for _, c in prof.values()),
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -442,7 +508,7 @@ def main(argv=None):
     else:
         rank, world, local = dist_setup()
         try:
-            res = run_ours(args, rank, world, local)
+            res = run_decode(args, local) if args.mode == "decode" else run_ours(args, rank, world, local)
         finally:
             if world > 1:
                 import torch.distributed as dist

@@ -182,9 +182,9 @@ absorbed_attn_kernel(const AbsParams p) {
     }
   } else if (warp == 1) {
     if (lane == 0 && n > 0) {
-      // ---------------- UMMA issuer. Order: S(0), S(1); then per block j:
-      // wait P(j), O += P(j) . C_j, release stage j, S(j+2) into S(j)'s
-      // buffer (the softmax has read S(j) before it wrote P(j)).
+      // ---------------- UMMA issuer: S(j) = Q K_j^T into S buffer j % 2, and
+      // O += P(j) . C_j once the softmax has written P(j), then release
+      // stage j (the scheduling rule is below).
       constexpr uint32_t idesc_qk = idesc_bf16_f32(64, 64, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(64, 256, 0, 1);
       const uint32_t stage0 = smem_u32(smem);
@@ -205,14 +205,7 @@ absorbed_attn_kernel(const AbsParams p) {
         ++commits;
         return true;
       };
-      bool ok = mbar_wait(bar(kAbsQReady), 0, ab, kErrWaitSoftmax);
-      if (ok) {
-        tc_fence_after();
-        ok = qk(0) && (n < 2 || qk(1));
-      }
-      for (int j = 0; j < n && ok; ++j) {
-        if (!(ok = mbar_wait(bar(kAbsPFull), j & 1, ab, kErrWaitSoftmax))) break;
-        tc_fence_after();
+      auto pv = [&](int j) {
         const uint32_t st = stage0 + (j % AbsSmem::K_STAGES) * AbsSmem::K_STAGE;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -226,7 +219,41 @@ absorbed_attn_kernel(const AbsParams p) {
         umma_commit(bar(kAbsPVDone));
         umma_commit(bar(kAbsKEmpty0 + j % AbsSmem::K_STAGES));
         ++commits;
-        if (j + 2 < n) ok = qk(j + 2);
+      };
+      bool ok = mbar_wait(bar(kAbsQReady), 0, ab, kErrWaitSoftmax);
+      if (ok) {
+        tc_fence_after();
+        ok = qk(0);
+      }
+      // Issue whichever is ready next: PV(next_pv) once the softmax has
+      // written P(next_pv), or S(next_qk) = Q K^T once its keys have landed
+      // and its S buffer is free (S(i-2)'s P handed over, i.e. PV(i-2)
+      // issued). In a fixed order a slow gather of block j+2 would hold back
+      // PV(j+1) behind it. Neither barrier can run two phases ahead: the
+      // softmax writes P(j+1) only after PV(j) completed, and the gather
+      // refills a stage only after the PV that read it.
+      int next_pv = 0, next_qk = 1;
+      uint64_t t_idle = 0;
+      while (ok && next_pv < n) {
+        if (next_qk < n && next_pv >= next_qk - 1 &&
+            mbar_test_wait(bar(kAbsKFull0 + next_qk % AbsSmem::K_STAGES), (next_qk / AbsSmem::K_STAGES) & 1)) {
+          ok = qk(next_qk);  // ready: returns at once
+          ++next_qk;
+          t_idle = 0;
+        } else if (mbar_test_wait(bar(kAbsPFull), next_pv & 1)) {
+          tc_fence_after();
+          pv(next_pv);
+          ++next_pv;
+          t_idle = 0;
+        } else {
+          const uint64_t now = global_timer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitTimeoutNs || ab.raised()) {
+            if (!ab.raised()) ab.raise(kErrWaitSoftmax);
+            ok = false;
+          }
+        }
       }
       if (ok) umma_commit(bar(kAbsODone));
       if (!ok && commits > 0) {

@@ -30,6 +30,7 @@ using Gemm2Kvb = mla::Gemm2Cfg<false>;  // latent x W_kvb^T  (B stored [N, K])
 using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as f16 for the attention
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
+using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
 
 // ------------------------------------------------------------------ device state
 
@@ -40,6 +41,7 @@ struct DeviceState {
   int pairs_kvb = 0;   // CTA pairs of the pair GEMMs that fit on the device at once
   int pairs_wo = 0;
   int pairs_unabs = 0;
+  int pairs_wo_narrow = 0;
   int* err = nullptr;  // address of g_mla_device_error on this device
 };
 
@@ -96,11 +98,14 @@ int device_state(DeviceState** out) {
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2KvbAttn::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2Unabs>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2Unabs::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_tc2_kernel<Gemm2WoNarrow>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm2WoNarrow::SMEM_BYTES) == cudaSuccess;
       if (ok) {
         st.pairs_kvb = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, Gemm2Kvb::SMEM_BYTES);
         st.pairs_wo = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, Gemm2Wo::SMEM_BYTES);
         st.pairs_unabs = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Unabs>, Gemm2Unabs::SMEM_BYTES);
-        ok = st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_unabs > 0;
+        st.pairs_wo_narrow = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2WoNarrow>, Gemm2WoNarrow::SMEM_BYTES);
+        ok = st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_unabs > 0 && st.pairs_wo_narrow > 0;
       }
       ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AbsSmem::BYTES) == cudaSuccess;
@@ -359,6 +364,10 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
       !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64) ||
       !map_2d(&tc, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
     return MLA_ERR_CUDA;
+  // With a single row tile (decode) the 256-wide tiles would leave most SMs
+  // idle while W_o streams through; 128-wide tiles double the pairs.
+  if (M <= Gemm2WoNarrow::BM)
+    return launch_gemm_pair<Gemm2WoNarrow>(ds->pairs_wo_narrow, ta, tb, tc, M, N, K, ds->err, 4, st);
   return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st);
 }
 

@@ -12,7 +12,9 @@ from .inputs import (  # noqa: F401
     D_ROPE,
     D_V,
     SOFTMAX_SCALE,
+    DecodeInputs,
     MlaInputs,
+    make_decode_inputs,
     make_inputs,
     make_topk,
     quantize_e4m3_block128,

@@ -197,6 +197,63 @@ def make_inputs(cfg, *, T: Optional[int] = None, B: Optional[int] = None,
                      name=c.get("name", ""))
 
 
+@dataclasses.dataclass
+class DecodeInputs:
+    B: int
+    T: int                         # cache length including the new position (s = T - 1)
+    H: int
+    topk: Optional[int]
+    fp8: bool
+    scale: float
+    q: torch.Tensor                # bf16 [B, H, 192] of the new position
+    kv_latent: torch.Tensor        # bf16 [B, T, 512] latent cache
+    k_pe: torch.Tensor             # bf16 [B, T, 64]
+    W_kvb: torch.Tensor
+    W_kvb_scale: Optional[torch.Tensor]
+    W_o: torch.Tensor
+    W_o_scale: Optional[torch.Tensor]
+    topk_idx: Optional[torch.Tensor]     # int32 [B, k]
+
+    def tensors(self):
+        return {k: v for k, v in dataclasses.asdict(self).items() if isinstance(v, torch.Tensor)}
+
+
+def make_decode_inputs(B: int, T: int, H: int, topk: Optional[int], seed: int, fp8: bool = False) -> DecodeInputs:
+    """One new position per sequence and its cache, with the distributions of
+    make_inputs (without the [B, T, H, 192] queries of the whole prefill).
+    The selection of the new query s = T - 1 follows the same rule: s itself
+    plus min(k, T) - 1 distinct positions of [0, s), in a shuffled order."""
+    g = lambda tid: _gen(seed, tid)  # noqa: E731
+    q = _randn_bf16((B, H, D_QK), g(_TID_Q))
+    lat = _randn_bf16((B, T, D_LATENT), g(_TID_LAT))
+    kpe = _randn_bf16((B, T, D_ROPE), g(_TID_KPE))
+    std_kvb = (1.0 / D_LATENT) ** 0.5
+    std_o = (1.0 / (H * D_V)) ** 0.5
+    if fp8:
+        wk, sk = quantize_e4m3_block128(_randn_f32((H * (D_NOPE + D_V), D_LATENT), g(_TID_WKVB), std_kvb),
+                                        g(_TID_SKVB))
+        wo, so = quantize_e4m3_block128(_randn_f32((H * D_V, D_MODEL), g(_TID_WO), std_o), g(_TID_SWO))
+    else:
+        wk = _randn_bf16((H * (D_NOPE + D_V), D_LATENT), g(_TID_WKVB), std_kvb)
+        wo = _randn_bf16((H * D_V, D_MODEL), g(_TID_WO), std_o)
+        sk = so = None
+    tk = None
+    if topk is not None:
+        gt = g(_TID_TOPK)
+        n = min(int(topk), T)
+        rows = []
+        for _ in range(B):
+            others = torch.randperm(T - 1, generator=gt)[: n - 1] if n > 1 else torch.empty(0, dtype=torch.int64)
+            sel = torch.cat([torch.tensor([T - 1]), others])
+            sel = sel[torch.randperm(n, generator=gt)]
+            if int(topk) > n:  # more entries than positions: out-of-range fillers select nothing
+                sel = torch.cat([sel, torch.arange(T, T + int(topk) - n)])
+            rows.append(sel)
+        tk = torch.stack(rows).to(torch.int32).contiguous()
+    return DecodeInputs(B=B, T=T, H=H, topk=topk, fp8=fp8, scale=SOFTMAX_SCALE, q=q, kv_latent=lat, k_pe=kpe,
+                        W_kvb=wk, W_kvb_scale=sk, W_o=wo, W_o_scale=so, topk_idx=tk)
+
+
 def sample_rows(B: int, T: int, k: Optional[int], n_random: int, seed: int,
                 batches=None) -> list:
     """Query rows (flattened b*T + s) for sampled parity: the sequence ends,
