@@ -60,6 +60,13 @@ struct AbsParams {
   const __nv_bfloat16* lat;    // kv_latent [B*T][512]
   const __nv_bfloat16* kpe;    // k_pe [B*T][64]
   __nv_bfloat16* olat;         // [rows][H][512]
+  // Split of each row's key list into `parts` contiguous runs of blocks, one
+  // CTA each (decode, where one CTA per row leaves most SMs idle). With
+  // parts > 1 a CTA writes its normalised partial output and its running
+  // max and sum instead of o_lat; absorbed_combine_kernel merges them.
+  int parts;
+  float2* part_ml;             // [rows][parts][H]: (max in the scaled log2 domain, sum)
+  __nv_bfloat16* part_o;       // [rows][parts][H][512]
   int* err;
 };
 
@@ -108,11 +115,17 @@ absorbed_attn_kernel(const AbsParams p) {
     return;
   }
   const int hgroups = (p.H + 63) >> 6;
-  const int row = static_cast<int>(blockIdx.x) / hgroups;  // query row of this launch
-  const int hh = static_cast<int>(blockIdx.x) % hgroups;   // group of 64 heads (slots past H compute zeros)
-  const int count = p.counts[row];
-  const int n = (count + 63) >> 6;                      // 64-key blocks
-  const int32_t* keys = p.lists + static_cast<int64_t>(row) * p.kpad;
+  const int row = static_cast<int>(blockIdx.x) / (hgroups * p.parts);  // query row of this launch
+  const int hh = static_cast<int>(blockIdx.x) / p.parts % hgroups;     // group of 64 heads (slots past H compute zeros)
+  const int part = static_cast<int>(blockIdx.x) % p.parts;
+  // This CTA's run of the row's 64-key blocks: [jb0, jb0 + n).
+  const int count_row = p.counts[row];
+  const int n_row = (count_row + 63) >> 6;
+  const int per_part = (n_row + p.parts - 1) / p.parts;
+  const int jb0 = part * per_part;
+  const int n = max(0, min(per_part, n_row - jb0));
+  const int count = n > 0 ? min(count_row - 64 * jb0, 64 * n) : 0;  // keys of this run
+  const int32_t* keys = p.lists + static_cast<int64_t>(row) * p.kpad + 64 * jb0;
   const int key_base = p.key_row0 + (row / p.rows_per_seq) * p.seq_stride;
 
   if (threadIdx.x == 0) {
@@ -395,8 +408,11 @@ absorbed_attn_kernel(const AbsParams p) {
     }
 
     if (ok) {
-      // lanes 0..15 write their head's o_lat row (512 bf16)
-      __nv_bfloat16* dst = p.olat + (static_cast<int64_t>(row) * p.H + hp) * 512;
+      // lanes 0..15 write their head's o_lat row (512 bf16), or with a split
+      // the run's normalised partial row; lanes 16..31 its (max, sum)
+      const int64_t prow = (static_cast<int64_t>(row) * p.parts + part) * p.H + hp;
+      __nv_bfloat16* dst = p.parts > 1 ? p.part_o + prow * 512 : p.olat + (static_cast<int64_t>(row) * p.H + hp) * 512;
+      if (p.parts > 1 && srow && hvalid) p.part_ml[prow] = make_float2(m_run, l_run);
       if (n > 0) {
         ok = warp_wait(bar(kAbsODone), 0, ab, kErrWaitMma);
         if (ok) {
@@ -420,7 +436,7 @@ absorbed_attn_kernel(const AbsParams p) {
         }
       } else if (!srow && hvalid) {
         uint4* d4 = reinterpret_cast<uint4*>(dst);
-        for (int i = 0; i < 64; ++i) d4[i] = make_uint4(0, 0, 0, 0);  // no selected key
+        for (int i = 0; i < 64; ++i) d4[i] = make_uint4(0, 0, 0, 0);  // no selected key (in this run)
       }
     }
   }
@@ -429,6 +445,53 @@ absorbed_attn_kernel(const AbsParams p) {
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// Merges the parts of a split row: per (row, head), with M the largest
+// part max, o_lat = sum_p w_p o_p / sum_p w_p where w_p = l_p 2^(m_p - M)
+// and o_p is part p's normalised output. One warp per (row, head), 16 of
+// the 512 values per lane. A head whose parts saw no key gets 0.
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(32 * kCombineWarps)
+absorbed_combine_kernel(const AbsParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);  // row * H + h
+  if (item >= static_cast<int64_t>(p.rows) * p.H) return;
+  const int64_t row = item / p.H, h = item % p.H;
+  float M = -INFINITY;
+  for (int q = 0; q < p.parts; ++q) M = fmaxf(M, p.part_ml[(row * p.parts + q) * p.H + h].x);
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  for (int q = 0; q < p.parts; ++q) {
+    const int64_t pr = (row * p.parts + q) * p.H + h;
+    const float2 ml = p.part_ml[pr];
+    const float w = ml.y > 0.f ? ml.y * ex2_approx(ml.x - M) : 0.f;
+    if (w == 0.f) continue;
+    wsum += w;
+    const uint4* src = reinterpret_cast<const uint4*>(p.part_o + pr * 512 + lane * 16);
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const uint4 u = __ldg(src + v);
+      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e]));
+        acc[8 * v + 2 * e] = fmaf(w, f.x, acc[8 * v + 2 * e]);
+        acc[8 * v + 2 * e + 1] = fmaf(w, f.y, acc[8 * v + 2 * e + 1]);
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(p.olat + item * 512 + lane * 16);
+#pragma unroll
+  for (int v = 0; v < 2; ++v)
+    dst[v] = make_uint4(pack_bf16x2(acc[8 * v] * inv, acc[8 * v + 1] * inv),
+                        pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv),
+                        pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv),
+                        pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv));
 }
 
 }  // namespace mla

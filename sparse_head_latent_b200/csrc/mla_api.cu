@@ -208,6 +208,8 @@ constexpr int64_t kMaxRows = int64_t(1) << 24;  // B*T limit (int32 tile coordin
 struct WsLayout {
   size_t kvh = kNone, attn = kNone, bitmap = kNone, blocks = kNone, wkvb = kNone, wo = kNone;
   size_t qabs = kNone, olat = kNone, lists = kNone, counts = kNone;  // absorbed path, one chunk of rows
+  size_t part_ml = kNone, part_o = kNone;  // decode: partial results of split rows
+  int parts = 1;                          // decode: CTAs per (sequence, 64-head group)
   int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
   int abs_chunk = 0;   // absorbed rows processed per pass
   int kpad = 0;        // pitch of the per-row key lists
@@ -218,6 +220,9 @@ struct WsLayout {
 // batch element, which bounds the workspace (q_abs and o_lat are
 // rows x H x 1 KB each).
 constexpr int kAbsChunkRows = 2048;
+// SM count the decode split is planned for (the workspace size cannot depend
+// on the device; a different count only changes how full the waves are).
+constexpr int kSmsForSplit = 148;
 // Cost model for MLA_PATH_AUTO: a tile group goes absorbed when its middle
 // row's causal prefix exceeds this many times the selection size. Measured
 // on B200 at T = 32768, H = 128, top-k 2048: the block-dense kernel costs
@@ -293,6 +298,18 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
     w.lists = take(B * static_cast<size_t>(w.kpad) * 4);
     w.counts = take(B * 4);
     w.attn = take(B * H * kDv * 2);
+    // Split each sequence's keys over several CTAs when B alone cannot fill
+    // the device: about two waves of CTAs, at least four 64-key blocks each.
+    const int hgroups = (d.H + 63) / 64;
+    const int want = (2 * kSmsForSplit + d.B * hgroups - 1) / (d.B * hgroups);
+    const int most = w.kpad / 64 / 4;
+    w.parts = want < most ? want : most;
+    if (w.parts > 16) w.parts = 16;
+    if (w.parts < 1) w.parts = 1;
+    if (w.parts > 1) {
+      w.part_ml = take(B * w.parts * H * 8);
+      w.part_o = take(B * w.parts * H * kL * 2);
+    }
   }
   const bool dec = entry == MLA_ENTRY_DECODE;
   if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
@@ -495,7 +512,8 @@ int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* ola
 int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const void* lat, const void* k_pe, int rows,
                               int key_row0, int rows_per_seq, int seq_stride, int kpad, const int32_t* lists,
                               const int32_t* counts, const void* qabs,
-                              const void* q_rows, void* olat, float scale, cudaStream_t st) {
+                              const void* q_rows, void* olat, float scale, cudaStream_t st, int parts = 1,
+                              void* part_ml = nullptr, void* part_o = nullptr) {
   mla::AbsParams p;
   p.rows = rows;
   p.H = d.H;
@@ -511,10 +529,19 @@ int launch_attention_absorbed(const DeviceState* ds, const mla_dims& d, const vo
   p.lat = static_cast<const __nv_bfloat16*>(lat);
   p.kpe = static_cast<const __nv_bfloat16*>(k_pe);
   p.olat = static_cast<__nv_bfloat16*>(olat);
+  p.parts = parts;
+  p.part_ml = static_cast<float2*>(part_ml);
+  p.part_o = static_cast<__nv_bfloat16*>(part_o);
   p.err = ds->err;
+  int rc = timed_launch(7, st, [&] {
+    mla::absorbed_attn_kernel<<<static_cast<unsigned>(rows * ((d.H + 63) / 64) * parts), mla::kAbsThreads,
+                                 mla::AbsSmem::BYTES, st>>>(p);
+  });
+  if (rc != MLA_OK || parts == 1) return rc;
+  const int64_t items = static_cast<int64_t>(rows) * d.H;
   return timed_launch(7, st, [&] {
-    mla::absorbed_attn_kernel<<<static_cast<unsigned>(rows * ((d.H + 63) / 64)), mla::kAbsThreads, mla::AbsSmem::BYTES,
-                                 st>>>(p);
+    mla::absorbed_combine_kernel<<<static_cast<unsigned>((items + mla::kCombineWarps - 1) / mla::kCombineWarps),
+                                    32 * mla::kCombineWarps, 0, st>>>(p);
   });
 }
 
@@ -635,7 +662,8 @@ int run_decode(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   if ((rc = launch_decode_lists(d, topk_idx, lay.kpad, lists, counts, st)) != MLA_OK) return rc;
   if ((rc = launch_gemm_absorb(ds, d.H, d.B, q, wk, qabs, st)) != MLA_OK) return rc;
   if ((rc = launch_attention_absorbed(ds, d, lat, k_pe, d.B, 0, 1, d.T, lay.kpad, lists, counts, qabs, q, olat, scale,
-                                      st)) != MLA_OK)
+                                      st, lay.parts, lay.parts > 1 ? ws_at(ws, lay.part_ml) : nullptr,
+                                      lay.parts > 1 ? ws_at(ws, lay.part_o) : nullptr)) != MLA_OK)
     return rc;
   if ((rc = launch_gemm_unabsorb(ds, d.H, d.B, olat, wk, attn, st)) != MLA_OK) return rc;
   const void* wo = W_o;

@@ -24,6 +24,10 @@ DECODE_CASES = {
     "fp8_weights": dict(B=2, T=200, H=2, topk=24, fp8=True),
     "every_position": dict(B=2, T=150, H=4, topk=None),
     "one_token_cache": dict(B=3, T=1, H=2, topk=4),
+    # few sequences and long selections: each query's keys are split over
+    # several CTAs and the partial results combined
+    "split_keys": dict(B=2, T=3000, H=4, topk=1024),
+    "split_keys_64_heads": dict(B=1, T=2100, H=64, topk=1024),
 }
 
 
@@ -69,3 +73,14 @@ def test_decode_sequence_without_a_valid_key_is_zero():
     assert not out[1].any()
     x.topk_idx[:, x.T - 1] = tk
     assert_close(out[:1].float().cpu().numpy(), _reference(x)[:1], "valid sequence")
+
+
+def test_decode_split_with_empty_parts():
+    # 1024 entries but about 300 distinct keys: the split is planned for 1024
+    # (four parts), so the last parts of the row receive no key at all.
+    x = synth.make_inputs(0, B=2, T=2000, H=4, topk=1024, seed=64)
+    tk = x.topk_idx[:, x.T - 1].clone()
+    tk = tk[:, :300].repeat(1, 4)[:, :1024].contiguous()
+    out = _decode(x, tk)
+    x.topk_idx[:, x.T - 1] = tk
+    assert_close(out.float().cpu().numpy(), _reference(x), "empty parts")
