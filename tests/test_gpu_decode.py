@@ -84,3 +84,48 @@ def test_decode_split_with_empty_parts():
     out = _decode(x, tk)
     x.topk_idx[:, x.T - 1] = tk
     assert_close(out.float().cpu().numpy(), _reference(x), "empty parts")
+
+
+def test_decode_replays_from_a_cuda_graph():
+    # The decode step only enqueues kernels on the given stream, so it can be
+    # captured once and replayed; the replay must reproduce the eager result
+    # bit for bit, also after the inputs change in place.
+    x = synth.make_inputs(0, B=4, T=2500, H=16, topk=512, seed=65)
+    g = {k: v.cuda() for k, v in x.tensors().items()}
+    T = x.T
+    q = g["q"][:, T - 1].contiguous()
+    tk = x.topk_idx[:, T - 1].contiguous().cuda()
+    dims = mla.make_dims(x.B, T, x.H, tk.shape[-1], False)
+    ws = torch.empty(mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_DECODE, True), dtype=torch.uint8, device="cuda")
+    out = torch.empty(x.B, 7168, dtype=torch.bfloat16, device="cuda")
+
+    def step(st=None):
+        mla.mla_decode(q, g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], topk_idx=tk, scale=x.scale,
+                       out=out, workspace=ws, stream=st)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    eager = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(torch.cuda.current_stream())
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert torch.equal(out, eager)
+    # new inputs written in place: the replay must agree with a fresh eager call
+    q.mul_(-1)
+    tk.copy_(torch.flip(tk, dims=[-1]) // 2)
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = out.clone()
+    step()
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert torch.equal(replayed, out)
+    assert not torch.equal(replayed, eager)
+    del graph
