@@ -6,9 +6,12 @@ import this package. The CUDA library never does.
 from .oracle import (  # noqa: F401
     attend_rows,
     build,
+    bf16_from_double,
     bf16_to_double,
+    e4m3_from_float,
     e4m3_to_double,
     prefill_rows,
     project_rows,
+    quantize_act,
     upproject_rows,
 )

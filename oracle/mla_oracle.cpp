@@ -28,6 +28,16 @@
 //     fp32 scale per 128 x 128 block of the stored [rows, cols] matrix.
 //   * W_kvb is stored [H*(dn+dv), L] (module [out, in]); W_o is stored
 //     [H*dv, D] (the math form o W_O).
+//   * Dynamic FP8 activations (Kimi K2 "Down projection" page, config.json
+//     quantization_config: activation_scheme "dynamic", fmt "e4m3", 128 x 128
+//     weight blocks), when act_e4m3 is set: the input of each FP8 linear layer
+//     -- the latent entering W_kvb and the attention output entering W_o -- is
+//     quantized per row in groups of 128 consecutive channels, s = amax / 448
+//     and code = e4m3(x / s), both divisions in fp32 rounding to nearest even,
+//     the conversion rounding to nearest even and saturating at +-448; an
+//     all-zero group gets s = 0. The layer then sees code * s. The attention
+//     output is a bf16 tensor in the pages' model, so it is rounded to bf16
+//     (nearest even) before it is quantized.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -60,6 +70,66 @@ double e4m3_value(uint8_t code) {
   return sign ? -mag : mag;
 }
 
+// bf16 value nearest to v (ties to an even last mantissa bit), as bits.
+// bf16 keeps fp32's 8 exponent bits and 7 of its mantissa bits.
+uint16_t bf16_bits_nearest(double v) {
+  double a = std::fabs(v);
+  double r = 0.0;
+  if (a != 0.0) {
+    int E = 0;
+    std::frexp(a, &E);        // a = f * 2^E, f in [0.5, 1)
+    int e = E - 1;            // a in [2^e, 2^(e+1))
+    if (e < -126) e = -126;   // subnormal range: fixed quantum
+    const double quantum = std::ldexp(1.0, e - 7);
+    r = std::nearbyint(a / quantum) * quantum;   // ties to even
+  }
+  const float f = static_cast<float>(std::signbit(v) ? -r : r);   // exact
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+// E4M3FN code nearest to x (ties to an even code), saturating at +-448.
+uint8_t e4m3_code_nearest(float x) {
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(x));
+  if (a == 0.0) return sign;
+  int E = 0;
+  std::frexp(a, &E);
+  int e = E - 1;
+  if (e < -6) e = -6;   // subnormals share the quantum of the smallest binade
+  const double quantum = std::ldexp(1.0, e - 3);
+  double v = std::nearbyint(a / quantum) * quantum;
+  if (v > 448.0) v = 448.0;
+  if (v == 0.0) return sign;
+  if (v < std::ldexp(1.0, -6)) return sign | static_cast<uint8_t>(v / std::ldexp(1.0, -9));
+  std::frexp(v, &E);
+  e = E - 1;
+  const int man = static_cast<int>((v / std::ldexp(1.0, e) - 1.0) * 8.0);
+  return sign | static_cast<uint8_t>(((e + 7) << 3) | man);
+}
+
+// One group of a row: codes[i] and the group's scale from x[0..n).
+void quantize_group(const float* x, int n, uint8_t* codes, float* scale) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) amax = std::fabs(x[i]) > amax ? std::fabs(x[i]) : amax;
+  const float s = amax / 448.0f;
+  *scale = s;
+  for (int i = 0; i < n; ++i) codes[i] = s == 0.0f ? 0 : e4m3_code_nearest(x[i] / s);
+}
+
+// Values a layer sees for an activation row under dynamic FP8: quantize the
+// row's groups of 128 channels and decode code * s.
+void fake_quantize_row(const float* x, int n, double* out) {
+  uint8_t codes[128];
+  float s = 0.0f;
+  for (int g = 0; g < n; g += 128) {
+    const int w = n - g < 128 ? n - g : 128;
+    quantize_group(x + g, w, codes, &s);
+    for (int i = 0; i < w; ++i) out[g + i] = e4m3_value(codes[i]) * static_cast<double>(s);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -79,10 +149,37 @@ struct mlao_problem {
   const float* W_o_scale;     // [H*d_v/128, d_model/128] when w_fp8
   const int32_t* topk_idx;    // [B,T,topk] or NULL (causal mask only)
   double scale;               // softmax scale
+  int act_e4m3;               // 1: dynamic per-token e4m3 activations into W_kvb and W_o
 };
 
 double mlao_bf16_to_double(uint16_t bits) { return bf16_value(bits); }
 double mlao_e4m3_to_double(uint8_t code) { return e4m3_value(code); }
+uint16_t mlao_bf16_from_double(double v) { return bf16_bits_nearest(v); }
+uint8_t mlao_e4m3_from_float(float x) { return e4m3_code_nearest(x); }
+
+// Dynamic activation quantization of x [rows][cols] (cols a multiple of 128):
+// codes [rows][cols], scales [rows][cols / 128].
+int mlao_quantize_act(const float* x, int rows, int cols, uint8_t* codes, float* scales) {
+  if (cols % 128 != 0) return 1;
+  for (int r = 0; r < rows; ++r)
+    for (int g = 0; g < cols / 128; ++g)
+      quantize_group(x + static_cast<size_t>(r) * cols + 128 * g, 128, codes + static_cast<size_t>(r) * cols + 128 * g,
+                     scales + static_cast<size_t>(r) * (cols / 128) + g);
+  return 0;
+}
+
+// Latent row at flattened position pos as the up-projection sees it.
+static void latent_row(const mlao_problem* p, int64_t pos, double* out) {
+  const int L = p->d_latent;
+  const uint16_t* lat = p->kv_latent + pos * L;
+  if (!p->act_e4m3) {
+    for (int j = 0; j < L; ++j) out[j] = bf16_value(lat[j]);
+    return;
+  }
+  std::vector<float> x(L);
+  for (int j = 0; j < L; ++j) x[j] = static_cast<float>(bf16_value(lat[j]));
+  fake_quantize_row(x.data(), L, out);
+}
 
 // Exact stored value of W_kvb[r][c] or W_o[r][c].
 static double weight_value(const void* w, const float* sc, int w_fp8, int cols,
@@ -106,12 +203,13 @@ int mlao_upproject_rows(const mlao_problem* p, int n_rows, const int64_t* rows, 
   for (int r = 0; r < R; ++r)
     for (int j = 0; j < L; ++j)
       wt[static_cast<size_t>(j) * R + r] = weight_value(p->W_kvb, p->W_kvb_scale, p->w_fp8, L, r, j);
+  std::vector<double> lat(L);
   for (int n = 0; n < n_rows; ++n) {
-    const uint16_t* lat = p->kv_latent + rows[n] * L;
+    latent_row(p, rows[n], lat.data());
     double* acc = kvh + static_cast<size_t>(n) * R;
     for (int r = 0; r < R; ++r) acc[r] = 0.0;
     for (int j = 0; j < L; ++j) {
-      const double a = bf16_value(lat[j]);
+      const double a = lat[j];
       const double* w = wt.data() + static_cast<size_t>(j) * R;
       for (int r = 0; r < R; ++r) acc[r] += a * w[r];
     }
@@ -153,7 +251,7 @@ int mlao_attend_rows(const mlao_problem* p, int n_rows, const int64_t* rows,
   std::vector<char> have;
   kv_cache.resize(static_cast<size_t>(p->B) * T * per_head);
   have.resize(static_cast<size_t>(p->B) * T);
-  std::vector<double> z, w;
+  std::vector<double> z, w, lat(L);
 
   for (int hi = 0; hi < n_heads; ++hi) {
     const int h = heads ? heads[hi] : hi;
@@ -178,10 +276,10 @@ int mlao_attend_rows(const mlao_problem* p, int n_rows, const int64_t* rows,
         const int64_t bt = b * T + A[a];
         double* kv = kv_cache.data() + static_cast<size_t>(bt) * per_head;
         if (!have[bt]) {  // k_nope_h[t] and v_h[t]
-          const uint16_t* lat = p->kv_latent + bt * L;
+          latent_row(p, bt, lat.data());
           for (int r = 0; r < per_head; ++r) kv[r] = 0.0;
           for (int j = 0; j < L; ++j) {
-            const double x = bf16_value(lat[j]);
+            const double x = lat[j];
             const double* wr = wt.data() + static_cast<size_t>(j) * per_head;
             for (int r = 0; r < per_head; ++r) kv[r] += x * wr[r];
           }
@@ -213,12 +311,20 @@ int mlao_attend_rows(const mlao_problem* p, int n_rows, const int64_t* rows,
 
 // Output projection of full-width attention rows:
 //   out[n][c] = sum_k attn[n][k] * W_o[k][c],  k = h*d_v + d ascending.
+// With act_e4m3 the row is first rounded to bf16 and quantized.
 int mlao_project_rows(const mlao_problem* p, int n_rows, const double* attn, double* out) {
   const int K = p->H * p->d_v, D = p->d_model;
+  std::vector<float> xb(K);
+  std::vector<double> xq(K);
   for (int n = 0; n < n_rows; ++n) {
     double* o = out + static_cast<size_t>(n) * D;
     for (int c = 0; c < D; ++c) o[c] = 0.0;
     const double* a = attn + static_cast<size_t>(n) * K;
+    if (p->act_e4m3) {
+      for (int k = 0; k < K; ++k) xb[k] = static_cast<float>(bf16_value(bf16_bits_nearest(a[k])));
+      fake_quantize_row(xb.data(), K, xq.data());
+      a = xq.data();
+    }
     for (int k = 0; k < K; ++k) {
       const double ak = a[k];
       if (!p->w_fp8) {

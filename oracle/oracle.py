@@ -41,6 +41,7 @@ class _Problem(ctypes.Structure):
         ("W_kvb", ctypes.c_void_p), ("W_kvb_scale", ctypes.c_void_p),
         ("W_o", ctypes.c_void_p), ("W_o_scale", ctypes.c_void_p),
         ("topk_idx", ctypes.c_void_p), ("scale", ctypes.c_double),
+        ("act_e4m3", ctypes.c_int),
     ]
 
 
@@ -59,6 +60,13 @@ def _load():
             lib.mlao_bf16_to_double.restype = ctypes.c_double
             lib.mlao_e4m3_to_double.argtypes = [ctypes.c_uint8]
             lib.mlao_e4m3_to_double.restype = ctypes.c_double
+            lib.mlao_bf16_from_double.argtypes = [ctypes.c_double]
+            lib.mlao_bf16_from_double.restype = ctypes.c_uint16
+            lib.mlao_e4m3_from_float.argtypes = [ctypes.c_float]
+            lib.mlao_e4m3_from_float.restype = ctypes.c_uint8
+            lib.mlao_quantize_act.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                              ctypes.c_void_p]
+            lib.mlao_quantize_act.restype = ctypes.c_int
             lib.mlao_upproject_rows.argtypes = [P, ctypes.c_int, i64p, dp]
             lib.mlao_attend_rows.argtypes = [P, ctypes.c_int, i64p, ctypes.c_int, i32p, dp]
             lib.mlao_project_rows.argtypes = [P, ctypes.c_int, dp, dp]
@@ -81,7 +89,7 @@ def _cpu(t):
 class _Bound:
     """Keeps the CPU tensors alive while the oracle reads them."""
 
-    def __init__(self, x, d_nope=128, d_rope=64, d_v=128, d_latent=512, d_model=None):
+    def __init__(self, x, d_nope=128, d_rope=64, d_v=128, d_latent=512, d_model=None, act_e4m3=False):
         self.keep = []
 
         def ptr(t):
@@ -112,6 +120,7 @@ class _Bound:
         p.W_o_scale = ptr(x.W_o_scale)
         p.topk_idx = ptr(tk.to(torch.int32) if tk is not None else None)
         p.scale = float(x.scale)
+        p.act_e4m3 = 1 if act_e4m3 else 0
         self.p = p
         self.H, self.d_v, self.d_model = H, d_v, d_model
         self.per_head = d_nope + d_v
@@ -122,7 +131,11 @@ def _rows_arr(rows):
 
 
 def upproject_rows(x, rows, **dims) -> np.ndarray:
-    """fp64 [n, H*(d_nope+d_v)]: latent rows times W_kvb (stored row order)."""
+    """fp64 [n, H*(d_nope+d_v)]: latent rows times W_kvb (stored row order).
+
+    Every entry point takes ``act_e4m3=True`` for dynamic FP8 activations: the
+    latent and the attention output are quantized per row in groups of 128
+    before W_kvb and W_o (see ``quantize_act``)."""
     lib = _load()
     bd = _Bound(x, **dims)
     r = _rows_arr(rows)
@@ -186,3 +199,25 @@ def bf16_to_double(bits: int) -> float:
 
 def e4m3_to_double(code: int) -> float:
     return _load().mlao_e4m3_to_double(int(code) & 0xFF)
+
+
+def bf16_from_double(v: float) -> int:
+    """bf16 bits of the value nearest to v (ties to even)."""
+    return int(_load().mlao_bf16_from_double(float(v)))
+
+
+def e4m3_from_float(v: float) -> int:
+    """E4M3FN code nearest to the fp32 value v (ties to even), saturating at +-448."""
+    return int(_load().mlao_e4m3_from_float(float(v)))
+
+
+def quantize_act(x):
+    """Dynamic activation quantization of x (float32 [rows, cols], cols % 128 == 0):
+    (codes uint8 [rows, cols], scales float32 [rows, cols // 128]), s = amax / 448 per group."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    rows, cols = a.shape
+    codes = np.zeros((rows, cols), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 128), dtype=np.float32)
+    rc = _load().mlao_quantize_act(a.ctypes.data, rows, cols, codes.ctypes.data, scales.ctypes.data)
+    assert rc == 0
+    return codes, scales

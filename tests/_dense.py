@@ -17,6 +17,19 @@ def dequant(w, scale):
     return codes * s
 
 
+def fake_quant_e4m3(x):
+    """Dynamic activation quantization restated with torch casts: per row, groups
+    of 128 channels, s = amax / 448 in float32, codes = float8_e4m3fn(x / s);
+    returns the float64 values code * s. x is float32 (or exactly convertible)."""
+    xf = x.to(torch.float32)
+    g = xf.reshape(*xf.shape[:-1], xf.shape[-1] // 128, 128)
+    s = g.abs().amax(-1, keepdim=True) / 448.0
+    safe = torch.where(s > 0, s, torch.ones_like(s))
+    codes = (g / safe).to(torch.float8_e4m3fn)
+    deq = codes.to(torch.float64) * s.to(torch.float64)
+    return deq.reshape(x.shape)
+
+
 def selection_matrix(B, T, topk_idx):
     """bool [B, T, T]: key t is selected for query s and t <= s."""
     allowed = torch.ones(T, T, dtype=torch.bool).tril()
@@ -30,13 +43,16 @@ def selection_matrix(B, T, topk_idx):
     return chosen[:, :, :T] & allowed
 
 
-def dense_block(x, topk_idx="inputs"):
-    """(attn fp64 [B, T, H, 128], out fp64 [B, T, 7168])."""
+def dense_block(x, topk_idx="inputs", act_e4m3=False):
+    """(attn fp64 [B, T, H, 128], out fp64 [B, T, 7168]). With act_e4m3 the latent
+    and the bf16-rounded attention output are fake-quantized before the projections."""
     B, T, H = x.B, x.T, x.H
     tk = x.topk_idx if isinstance(topk_idx, str) else topk_idx
     wk = dequant(x.W_kvb, x.W_kvb_scale)
     wo = dequant(x.W_o, x.W_o_scale)
     latent = x.kv_latent.to(torch.float64)
+    if act_e4m3:
+        latent = fake_quant_e4m3(x.kv_latent.to(torch.float32))
     up = torch.matmul(latent, wk.t()).reshape(B, T, H, 256)
     k_nope, v = up[..., :128], up[..., 128:]
     rope = x.k_pe.to(torch.float64).unsqueeze(2).expand(B, T, H, 64)
@@ -50,5 +66,8 @@ def dense_block(x, topk_idx="inputs"):
     probs = torch.softmax(logits, dim=-1)
     probs = torch.nan_to_num(probs, nan=0.0)                      # empty rows -> 0
     attn = torch.matmul(probs, vh).permute(0, 2, 1, 3).contiguous()  # [B, T, H, 128]
-    out = torch.matmul(attn.reshape(B, T, H * 128), wo)
+    a = attn.reshape(B, T, H * 128)
+    if act_e4m3:
+        a = fake_quant_e4m3(a.to(torch.bfloat16).to(torch.float32))
+    out = torch.matmul(a, wo)
     return attn, out

@@ -42,6 +42,20 @@ MUTANTS = [
     ("bf16_shift", [("static_cast<uint32_t>(bits) << 16;", "static_cast<uint32_t>(bits) << 15;")]),
     ("fp8_scale_transposed", [("sc[(r / 128) * sc_cols + (c / 128)]", "sc[(c / 128) % sc_cols + (r / 128) % 2]")]),
     ("empty_row_not_zero", [("if (A.empty()) continue;  // no surviving key: attn = 0", "")]),
+    # dynamic FP8 activations
+    ("act_scale_447", [("const float s = amax / 448.0f;", "const float s = amax / 447.0f;")]),
+    ("act_ties_away", [("double v = std::nearbyint(a / quantum) * quantum;",
+                        "double v = std::round(a / quantum) * quantum;")]),
+    ("act_no_saturation", [("if (v > 448.0) v = 448.0;", "")]),
+    ("act_subnormal_quantum", [("if (e < -6) e = -6;", "if (e < -7) e = -7;")]),
+    ("act_group_64", [("const int w = n - g < 128 ? n - g : 128;", "const int w = n - g < 64 ? n - g : 64;"),
+                      ("for (int g = 0; g < n; g += 128) {", "for (int g = 0; g < n; g += 64) {")]),
+    ("act_latent_not_quantized", [("  if (!p->act_e4m3) {\n    for (int j = 0; j < L; ++j) out[j] = bf16_value(lat[j]);",
+                                   "  if (true) {\n    for (int j = 0; j < L; ++j) out[j] = bf16_value(lat[j]);")]),
+    ("act_attn_not_rounded", [("xb[k] = static_cast<float>(bf16_value(bf16_bits_nearest(a[k])));",
+                               "xb[k] = static_cast<float>(a[k]);")]),
+    ("bf16_round_quantum", [("const double quantum = std::ldexp(1.0, e - 7);",
+                             "const double quantum = std::ldexp(1.0, e - 8);")]),
 ]
 
 
@@ -66,8 +80,17 @@ def _run_pins(so):
     return r.returncode
 
 
+# Scratch for the mutant builds, inside the repository's ignored build folder.
+SCRATCH = os.path.join(ROOT, "_build")
+
+
+def _scratch():
+    os.makedirs(SCRATCH, exist_ok=True)
+    return tempfile.mkdtemp(prefix="mla_mutants_", dir=SCRATCH)
+
+
 def test_every_mutant_is_caught():
-    tmp = tempfile.mkdtemp(prefix="mla_mutants_")
+    tmp = _scratch()
     try:
         libs = [(n, _build_mutant(tmp, n, e)) for n, e in MUTANTS]
         with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
@@ -79,7 +102,7 @@ def test_every_mutant_is_caught():
 
 
 def test_unmutated_copy_passes():
-    tmp = tempfile.mkdtemp(prefix="mla_mutants_")
+    tmp = _scratch()
     try:
         so = _build_mutant(tmp, "identity", [])
         assert _run_pins(so) == 0

@@ -10,7 +10,13 @@ to an invariant of the method, or to a library routine on a special case:
   * a single selected key returns that key's value vector exactly;
   * q = 0 returns the mean of the selected value vectors;
   * the order of top-k entries and duplicate entries change nothing;
-  * out-of-range top-k entries select nothing.
+  * out-of-range top-k entries select nothing;
+  * dynamic FP8 activations: the e4m3 encoder returns the nearest code (brute
+    force over the format's table, ties to even, saturating at 448) and agrees
+    with torch's float8_e4m3fn cast; the group scale is amax / 448 and the
+    largest element maps to +-448; quantization commutes with powers of two;
+    the quantized projections equal fp64 matmuls of the dequantized rows and
+    the whole block equals the dense restatement with torch's casts.
 """
 import math
 import os
@@ -22,7 +28,7 @@ import torch.nn.functional as F
 
 import oracle
 import synth
-from tests._dense import dense_block, dequant
+from tests._dense import dense_block, dequant, fake_quant_e4m3
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -280,3 +286,151 @@ def test_scores_scale_enters_linearly():
     x.scale = synth.SOFTMAX_SCALE
     a2 = oracle.attend_rows(x, _all_rows(x))
     assert _rel(a1, a2) < 1e-14
+
+
+# ---------------------------------------------------------------- dynamic FP8 activations
+
+def _e4m3_values():
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _e4m3_probe_values(seed=21):
+    """float32 values in [-448, 448]: random magnitudes over the whole range
+    plus every midpoint between neighbouring codes (the ties)."""
+    vals = _e4m3_values()
+    pos = np.unique(vals[(vals >= 0) & ~np.isnan(vals)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(seed)
+    rand = rng.standard_normal(4000) * 10.0 ** rng.uniform(-4, 2.6, 4000)
+    xs = np.concatenate([rand, mids, -mids, pos, -pos, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20)])
+    xs = xs.astype(np.float32)
+    return xs[np.abs(xs) <= 448]
+
+
+def test_e4m3_encode_is_the_nearest_code():
+    vals = _e4m3_values()
+    finite = ~np.isnan(vals)
+    for x in _e4m3_probe_values():
+        c = oracle.e4m3_from_float(float(x))
+        sign = 0x80 if np.signbit(x) else 0
+        cand = np.array([k for k in range(256) if finite[k] and (k & 0x80) == sign])
+        d = np.abs(vals[cand] - np.float64(x))
+        best = cand[d == d.min()]
+        if len(best) > 1:  # a tie: the code with an even mantissa
+            best = best[(best & 1) == 0]
+        assert c == int(best[0]), (x, c, best)
+
+
+def test_e4m3_encode_matches_torch_cast():
+    xs = _e4m3_probe_values(seed=22)
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([oracle.e4m3_from_float(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(mine, ref)
+
+
+def test_e4m3_encode_saturates_at_448():
+    for v in (448.0, 448.5, 463.9, 464.0, 480.0, 1.0e6, 3.0e38):
+        assert oracle.e4m3_from_float(v) == 0x7E
+        assert oracle.e4m3_from_float(-v) == 0xFE
+    assert oracle.e4m3_from_float(2.0 ** -10) == 0x00       # tie between 0 and 2^-9
+    assert oracle.e4m3_from_float(3 * 2.0 ** -10) == 0x02   # tie between 2^-9 and 2^-8
+
+
+def test_bf16_rounding_is_nearest_and_matches_torch():
+    rng = np.random.default_rng(23)
+    f32 = (rng.standard_normal(3000) * 10.0 ** rng.uniform(-30, 30, 3000)).astype(np.float32)
+    ref = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    mine = np.array([oracle.bf16_from_double(float(v)) for v in f32], dtype=np.uint16)
+    assert np.array_equal(mine, ref)
+    for v in rng.standard_normal(500) * 10.0 ** rng.uniform(-5, 5, 500):
+        b = oracle.bf16_from_double(float(v))
+        got = oracle.bf16_to_double(b)
+        lo, hi = oracle.bf16_to_double(b - 1), oracle.bf16_to_double(b + 1)
+        assert abs(got - v) <= abs(lo - v) and abs(got - v) <= abs(hi - v)
+
+
+def _act_rows(seed=24, rows=6, cols=384):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)) * 10.0 ** rng.uniform(-3, 3, (rows, 1))
+    x = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    x[1, 128:256] = 0.0          # an all-zero group
+    x[2, :128] = 0.0
+    x[2, 17] = -3.5              # a group with a single non-zero element
+    return x
+
+
+def test_act_quantization_closed_forms():
+    x = _act_rows()
+    codes, s = oracle.quantize_act(x)
+    g = x.reshape(x.shape[0], -1, 128)
+    amax = np.abs(g).max(-1)
+    assert np.array_equal(s, amax / np.float32(448.0))
+    vals = _e4m3_values()
+    deq = vals[codes].reshape(g.shape) * s[..., None].astype(np.float64)
+    cg = codes.reshape(g.shape)
+    for r in range(g.shape[0]):
+        for j in range(g.shape[1]):
+            if amax[r, j] == 0:
+                assert s[r, j] == 0 and not cg[r, j].any()
+                continue
+            i = int(np.argmax(np.abs(g[r, j])))
+            assert cg[r, j, i] in (0x7E, 0xFE)
+            y = np.abs(g[r, j].astype(np.float64)) / np.float64(s[r, j])
+            e = np.floor(np.log2(np.maximum(y, 2.0 ** -30)))
+            half_ulp = 2.0 ** (np.maximum(e, -6) - 4)
+            bound = (half_ulp + y * 2.0 ** -23) * np.float64(s[r, j])
+            assert np.all(np.abs(deq[r, j] - g[r, j]) <= bound)
+    assert deq[2, 0, 17] == -3.5
+
+
+def test_act_quantization_commutes_with_powers_of_two():
+    x = _act_rows(seed=25)
+    c0, s0 = oracle.quantize_act(x)
+    c1, s1 = oracle.quantize_act(x * np.float32(2.0 ** 7))
+    assert np.array_equal(c0, c1) and np.array_equal(s1, s0 * np.float32(2.0 ** 7))
+
+
+def test_act_quantization_matches_torch_casts():
+    x = _act_rows(seed=26, rows=9)
+    codes, s = oracle.quantize_act(x)
+    deq = _e4m3_values()[codes] * np.repeat(s.astype(np.float64), 128, axis=1)
+    ref = fake_quant_e4m3(torch.from_numpy(x)).numpy()
+    assert np.array_equal(deq, ref)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_act_e4m3_upprojection_equals_matmul_of_dequantized_latent(fp8):
+    x = _tiny(B=2, T=20, H=2, fp8=fp8)
+    rows = [0, 7, 19, 20, 39]
+    got = oracle.upproject_rows(x, rows, act_e4m3=True)
+    lat = x.kv_latent.reshape(-1, 512).to(torch.float32)[rows].numpy()
+    codes, s = oracle.quantize_act(lat)
+    deq = torch.from_numpy(_e4m3_values()[codes] * np.repeat(s.astype(np.float64), 128, axis=1))
+    ref = (deq @ dequant(x.W_kvb, x.W_kvb_scale).t()).numpy()
+    assert _rel(got, ref) < 1e-13
+    assert _rel(got, oracle.upproject_rows(x, rows)) > 1e-4   # the quantization is applied
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_act_e4m3_projection_equals_matmul_of_dequantized_rows(fp8):
+    x = _tiny(H=2, fp8=fp8)
+    g = torch.Generator().manual_seed(12)
+    attn = torch.randn(5, 2 * 128, generator=g, dtype=torch.float64)
+    got = oracle.project_rows(x, attn.numpy(), act_e4m3=True)
+    rounded = attn.to(torch.bfloat16).to(torch.float32).numpy()
+    codes, s = oracle.quantize_act(rounded)
+    deq = torch.from_numpy(_e4m3_values()[codes] * np.repeat(s.astype(np.float64), 128, axis=1))
+    ref = (deq @ dequant(x.W_o, x.W_o_scale)).numpy()
+    assert _rel(got, ref) < 1e-13
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_act_e4m3_block_equals_dense_restatement(fp8):
+    x = _tiny(B=2, T=40, H=2, topk=10, fp8=fp8)
+    attn, out = oracle.prefill_rows(x, _all_rows(x), act_e4m3=True)
+    ref_attn, ref_out = dense_block(x, act_e4m3=True)
+    assert _rel(attn, ref_attn.reshape(-1, 2, 128).numpy()) < 1e-12
+    assert _rel(out, ref_out.reshape(-1, 7168).numpy()) < 1e-12
+    _, out_bf16 = oracle.prefill_rows(x, _all_rows(x))
+    d = np.linalg.norm(out - out_bf16) / np.linalg.norm(out_bf16)
+    assert 1e-3 < d < 0.1   # e4m3 activations move the output by about a percent
