@@ -40,7 +40,8 @@ import synth  # noqa: E402
 METRIC = "sparse MLA prefill TFLOP/s and queries/s (T=4096,H=128,top-k 2048); % of bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "attn.cuh", "attn_abs.cuh", "prepass.cuh", "dequant.cuh", "mla_api.cu")
+KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "quant.cuh", "attn.cuh", "attn_abs.cuh", "prepass.cuh",
+                  "dequant.cuh", "mla_api.cu")
 
 
 def parse_args(argv=None):
@@ -59,6 +60,8 @@ def parse_args(argv=None):
     p.add_argument("--T", type=int, default=None, help="override the workload's sequence length")
     p.add_argument("--H", type=int, default=None, help="override the workload's head count")
     p.add_argument("--topk", type=int, default=None, help="override the workload's top-k")
+    p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
+                   help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
     return p.parse_args(argv)
 
 
@@ -288,7 +291,10 @@ def run_ours(args, rank, world, local):
     wm = work_model(x)
     dev = torch.device("cuda", local)
     g = {k: v.to(dev) for k, v in x.tensors().items()}
-    dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8)
+    act = mla.MLA_ACT_E4M3_DYNAMIC if args.act == "e4m3" else mla.MLA_ACT_BF16
+    if act and not x.fp8:
+        raise SystemExit("--act e4m3 needs a workload with e4m3 weights (--config 4)")
+    dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8, act=act)
     ws_bytes = mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_PREFILL, x.topk_idx is not None)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = torch.empty(x.B, x.T, 7168, dtype=torch.bfloat16, device=dev)
@@ -297,7 +303,7 @@ def run_ours(args, rank, world, local):
     def step():
         mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g.get("W_kvb_scale"),
                         g.get("W_o_scale"), topk_idx=g.get("topk_idx"), scale=x.scale, out=out,
-                        workspace=ws, stream=stream)
+                        workspace=ws, stream=stream, act=act)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -335,7 +341,7 @@ def run_ours(args, rank, world, local):
     d2h = host_out.numel() * host_out.element_size()
     pipe = mla.PrefillPipeline(x.B, x.T, x.H, g["W_kvb"], g["W_o"], g.get("W_kvb_scale"), g.get("W_o_scale"),
                                topk=x.topk_idx.shape[-1] if x.topk_idx is not None else None, scale=x.scale,
-                               device=dev)
+                               device=dev, act=act)
     for _ in range(3):
         pipe.submit(host_in, host_out)
     pipe.synchronize()
@@ -378,15 +384,22 @@ def run_ours(args, rank, world, local):
     dom_avg_ms = prof[dom][0] / prof[dom][1]
     achieved = kflops[dom] / (dom_avg_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
+    # With e4m3 activations the projections are e4m3 x e4m3 contractions: their
+    # peak is the measured bf16 peak times the nominal fp8 / bf16 ratio (2).
+    dom_fp8 = act and dom in ("gemm_kvb", "gemm_wo")
+    dom_peak = 2 * peak if dom_fp8 else peak
     roof_t = max(wm["flops"] / (peak * 1e12), wm["compulsory_bytes"] / (peaks["hbm_gbs"] * 1e9))
     clk = clocks.summary(t_wall0, t_wall2)
     result = {
         "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 projections, bf16 attention" if act else "bf16",
         "data": "synthetic (seeded; shapes and distributions of the workload; no checkpoint)",
         "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
-                   "weights": "e4m3 block-128" if x.fp8 else "bf16", "parallelism": f"independent sequences x{world}",
+                   "weights": "e4m3 block-128" if x.fp8 else "bf16",
+                   "activations": "e4m3 dynamic 1x128" if act else "bf16",
+                   "parallelism": f"independent sequences x{world}",
                    "l2": "no flush: every step reads > 600 MB, inputs larger than the 126 MB L2"},
         "queries_per_s": round(qps, 1),
         "frac_of_bf16_peak": round(tflops / world / peak, 4),
@@ -394,10 +407,11 @@ def run_ours(args, rank, world, local):
         "algorithmic_gflop_per_step": round(wm["flops"] / 1e9, 2),
         "selected_pairs": wm["pairs"],
         "per_kernel": per_kernel,
-        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic(dom, name),
-                     "peak_source": f"{peak_src} bf16 dense (burst), MEASURED_PEAKS.json"},
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": dom_peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / dom_peak, 4),
+                     "traffic": ncu_traffic(dom, name + ("_act8" if act else "")),
+                     "peak_source": (f"{peak_src} bf16 dense (burst) x 2 (nominal e4m3/bf16 ratio), MEASURED_PEAKS.json"
+                                     if dom_fp8 else f"{peak_src} bf16 dense (burst), MEASURED_PEAKS.json")},
         "e2e": {"value": round(e2e_tflops, 2), "unit": UNIT, "h2d_bytes_per_step": h2d * world,
                 "d2h_bytes_per_step": d2h * world, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": int(sum(n for _, n in prof.values())),

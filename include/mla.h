@@ -71,12 +71,28 @@ typedef enum {
   MLA_PATH_ABSORBED = 2      /* every row with a topk_idx: absorbed form over the gathered keys */
 } mla_path;
 
+/* Activations entering the two projections (W_kvb, W_o).
+ * MLA_ACT_E4M3_DYNAMIC follows the Kimi K2 "Down projection" page's
+ * quantization_config (activation_scheme "dynamic", fmt "e4m3", 128 x 128
+ * weight blocks): the latent rows entering W_kvb and the attention rows
+ * entering W_o are quantized on the fly per row and group of 128 channels
+ * (see mla_quantize_act) and the projections run as e4m3 x e4m3 tensor-core
+ * GEMMs with the activation and weight block scales applied per 128-deep K
+ * block. Needs wdtype MLA_W_E4M3_BLOCK128 and the block-dense attention path
+ * (MLA_PATH_AUTO then means block-dense; MLA_PATH_ABSORBED and mla_decode
+ * return MLA_ERR_UNSUPPORTED). */
+typedef enum {
+  MLA_ACT_BF16 = 0,          /* bf16 activations (weights dequantized for e4m3) */
+  MLA_ACT_E4M3_DYNAMIC = 1   /* dynamic per-token 1 x 128 e4m3 activations */
+} mla_act;
+
 typedef struct {
   int B, T, H;
   int d_nope, d_rope, d_v, d_latent, d_model;
   int topk;          /* entries per row of topk_idx (ignored when topk_idx == NULL) */
   mla_wdtype wdtype; /* storage of W_kvb and W_o */
   mla_path path;     /* MLA_PATH_AUTO (0) unless a caller forces one path */
+  mla_act act;       /* MLA_ACT_BF16 (0) unless the activations are quantized */
 } mla_dims;
 
 /* Entry points, for mla_workspace_bytes(). */
@@ -99,7 +115,9 @@ size_t mla_workspace_bytes(const mla_dims* dims, int entry, int has_topk);
  *               i < 128 and v_h[i-128] otherwise
  *   W_kvb_scale: fp32 [2H, 4] (block scales) for e4m3, else ignored
  *   kvh_out   : bf16 [B*T, H*256], same column order as W_kvb's rows
- * Uses the tcgen05 tensor-core GEMM; fp32 accumulation, bf16 rounding. */
+ * Uses the tcgen05 tensor-core GEMM; fp32 accumulation, bf16 rounding.
+ * With dims->act = MLA_ACT_E4M3_DYNAMIC the latent is quantized first and
+ * the GEMM is e4m3 x e4m3 (kind::f8f6f4) with per-block scales. */
 int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_kvb,
                      const float* W_kvb_scale, void* kvh_out, void* workspace,
                      size_t ws_bytes, mla_stream_t stream);
@@ -211,6 +229,20 @@ int mla_attend_static(const mla_dims* dims, const void* q, const void* kv_latent
                       const int32_t* topk_idx, float scale, void* attn_out,
                       mla_stream_t stream);
 
+/* Dynamic activation quantization (the step MLA_ACT_E4M3_DYNAMIC runs in
+ * front of each projection), exposed on its own.
+ *   x      : bf16 [rows, cols], cols a multiple of 128 (row pitch cols)
+ *   codes  : e4m3 [rows, cols]: code = e4m3(x / s), the division in fp32 and
+ *            the conversion rounding to nearest even, saturating at +-448
+ *   scales : fp32 [cols / 128, rows]: s = amax / 448 (fp32, nearest even) of
+ *            each row's group of 128 columns; an all-zero group gets s = 0
+ *            and zero codes. Group-major so that one group's row scales are
+ *            contiguous.
+ * x, codes and scales must be 16-byte aligned. Stream-ordered, no
+ * workspace. Errors: MLA_ERR_NULL, MLA_ERR_SHAPE (rows < 0, cols not a
+ * positive multiple of 128), MLA_ERR_ALIGN, MLA_ERR_CUDA. */
+int mla_quantize_act(const void* x, int rows, int cols, void* codes, float* scales, mla_stream_t stream);
+
 /* Human-readable text of a status code (static storage). */
 const char* mla_status_str(int status);
 
@@ -227,9 +259,9 @@ int mla_device_status(mla_stream_t stream, int* device_error);
  * milliseconds and launch count, then stops recording.
  * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention
  * (block-dense), 4 W_o GEMM, 5 per-row key lists (prefill and decode),
- * 6 absorb and un-absorb GEMMs, 7 attention (absorbed). Arrays must hold MLA_PROFILE_CLASSES
- * entries. */
-#define MLA_PROFILE_CLASSES 8
+ * 6 absorb and un-absorb GEMMs, 7 attention (absorbed), 8 activation
+ * quantization. Arrays must hold MLA_PROFILE_CLASSES entries. */
+#define MLA_PROFILE_CLASSES 9
 int mla_profile_begin(void);
 int mla_profile_end(float* ms_total, int* launches);
 

@@ -314,25 +314,29 @@ int mlao_attend_rows(const mlao_problem* p, int n_rows, const int64_t* rows,
 // With act_e4m3 the row is first rounded to bf16 and quantized.
 int mlao_project_rows(const mlao_problem* p, int n_rows, const double* attn, double* out) {
   const int K = p->H * p->d_v, D = p->d_model;
+  // The rows as W_o sees them (quantized when act_e4m3).
+  std::vector<double> rows_in(static_cast<size_t>(n_rows) * K);
   std::vector<float> xb(K);
-  std::vector<double> xq(K);
   for (int n = 0; n < n_rows; ++n) {
-    double* o = out + static_cast<size_t>(n) * D;
-    for (int c = 0; c < D; ++c) o[c] = 0.0;
     const double* a = attn + static_cast<size_t>(n) * K;
+    double* r = rows_in.data() + static_cast<size_t>(n) * K;
     if (p->act_e4m3) {
       for (int k = 0; k < K; ++k) xb[k] = static_cast<float>(bf16_value(bf16_bits_nearest(a[k])));
-      fake_quantize_row(xb.data(), K, xq.data());
-      a = xq.data();
+      fake_quantize_row(xb.data(), K, r);
+    } else {
+      for (int k = 0; k < K; ++k) r[k] = a[k];
     }
-    for (int k = 0; k < K; ++k) {
-      const double ak = a[k];
-      if (!p->w_fp8) {
-        const uint16_t* wr = static_cast<const uint16_t*>(p->W_o) + static_cast<size_t>(k) * D;
-        for (int c = 0; c < D; ++c) o[c] += ak * bf16_value(wr[c]);
-      } else {
-        for (int c = 0; c < D; ++c) o[c] += ak * weight_value(p->W_o, p->W_o_scale, 1, D, k, c);
-      }
+  }
+  for (size_t i = 0; i < static_cast<size_t>(n_rows) * D; ++i) out[i] = 0.0;
+  // Each W_o row is decoded once and applied to every row; every output
+  // still sums over k in ascending order.
+  std::vector<double> w(D);
+  for (int k = 0; k < K; ++k) {
+    for (int c = 0; c < D; ++c) w[c] = weight_value(p->W_o, p->W_o_scale, p->w_fp8, D, k, c);
+    for (int n = 0; n < n_rows; ++n) {
+      const double ak = rows_in[static_cast<size_t>(n) * K + k];
+      double* o = out + static_cast<size_t>(n) * D;
+      for (int c = 0; c < D; ++c) o[c] += ak * w[c];
     }
   }
   return 0;

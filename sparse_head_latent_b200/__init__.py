@@ -8,6 +8,8 @@ This package is its thin ctypes binding; the library is loaded on first
 use and a missing build is an error, never a fallback.
 """
 from .mla import (  # noqa: F401
+    MLA_ACT_BF16,
+    MLA_ACT_E4M3_DYNAMIC,
     MLA_ENTRY_ATTEND,
     MLA_ENTRY_DECODE,
     MLA_ENTRY_KV_UPPROJECT,
@@ -31,6 +33,7 @@ from .mla import (  # noqa: F401
     mla_prefill,
     mla_profile_begin,
     mla_profile_end,
+    mla_quantize_act,
     mla_status_str,
     mla_workspace_bytes,
 )

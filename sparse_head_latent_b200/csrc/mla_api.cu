@@ -17,7 +17,9 @@
 #include "attn_abs.cuh"
 #include "dequant.cuh"
 #include "gemm2.cuh"
+#include "gemm8.cuh"
 #include "prepass.cuh"
+#include "quant.cuh"
 #include "ptx.cuh"
 
 // Device error word: kernels record the first error code here.
@@ -31,6 +33,9 @@ using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as 
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
 using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
+using Gemm8Kvb = mla::Gemm8Cfg<false>;         // e4m3 latent x e4m3 W_kvb^T
+using Gemm8KvbAttn = mla::Gemm8Cfg<false, true>;  // same, v tiles written as f16 for the attention
+using Gemm8Wo = mla::Gemm8Cfg<true>;           // e4m3 attn x e4m3 W_o (B stored [K, N])
 
 // ------------------------------------------------------------------ device state
 
@@ -42,11 +47,13 @@ struct DeviceState {
   int pairs_wo = 0;
   int pairs_unabs = 0;
   int pairs_wo_narrow = 0;
+  int pairs8_kvb = 0;  // CTA pairs of the e4m3 GEMMs
+  int pairs8_wo = 0;
   int* err = nullptr;  // address of g_mla_device_error on this device
 };
 
 template <class Kernel>
-int max_pairs(Kernel k, int smem) {
+int max_pairs(Kernel k, int smem, int threads = 192) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -54,7 +61,7 @@ int max_pairs(Kernel k, int smem) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -107,6 +114,17 @@ int device_state(DeviceState** out) {
         st.pairs_wo_narrow = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2WoNarrow>, Gemm2WoNarrow::SMEM_BYTES);
         ok = st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_unabs > 0 && st.pairs_wo_narrow > 0;
       }
+      ok = ok && cudaFuncSetAttribute(mla::gemm_e4m3_tc2_kernel<Gemm8Kvb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Gemm8Kvb::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_e4m3_tc2_kernel<Gemm8KvbAttn>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Gemm8KvbAttn::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_e4m3_tc2_kernel<Gemm8Wo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Gemm8Wo::SMEM_BYTES) == cudaSuccess;
+      if (ok) {
+        st.pairs8_kvb = max_pairs(mla::gemm_e4m3_tc2_kernel<Gemm8Kvb>, Gemm8Kvb::SMEM_BYTES, Gemm8Kvb::THREADS);
+        st.pairs8_wo = max_pairs(mla::gemm_e4m3_tc2_kernel<Gemm8Wo>, Gemm8Wo::SMEM_BYTES, Gemm8Wo::THREADS);
+        ok = st.pairs8_kvb > 0 && st.pairs8_wo > 0;
+      }
       ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AbsSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -132,14 +150,14 @@ int device_state(DeviceState** out) {
 // Row-major bf16/u8 matrix [outer, inner] with a row pitch; box
 // [box_outer, box_inner]; 128-byte swizzle; out-of-range rows read as zero.
 bool map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-            uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+            uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {pitch_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
-  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 tensor [B, T, inner] (row pitch inner*2 bytes), box [1, box_rows, 64];
@@ -209,6 +227,8 @@ struct WsLayout {
   size_t kvh = kNone, attn = kNone, bitmap = kNone, blocks = kNone, wkvb = kNone, wo = kNone;
   size_t qabs = kNone, olat = kNone, lists = kNone, counts = kNone;  // absorbed path, one chunk of rows
   size_t part_ml = kNone, part_o = kNone;  // decode: partial results of split rows
+  size_t lat8 = kNone, lat8_s = kNone;    // e4m3 activations: quantized latent and its scales
+  size_t attn8 = kNone, attn8_s = kNone;  // e4m3 activations: quantized attention rows and scales
   int parts = 1;                          // decode: CTAs per (sequence, 64-head group)
   int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
   int abs_chunk = 0;   // absorbed rows processed per pass
@@ -236,7 +256,7 @@ constexpr int kAbsorbRatio = 11;
 int absorbed_first_group(const mla_dims& d, bool has_topk) {
   const int nq = (d.T + 127) / 128;
   const int ng = (nq + 3) / 4;
-  if (!has_topk || d.path == MLA_PATH_BLOCK_DENSE) return ng;
+  if (!has_topk || d.path == MLA_PATH_BLOCK_DENSE || d.act == MLA_ACT_E4M3_DYNAMIC) return ng;
   if (d.path == MLA_PATH_ABSORBED) return 0;
   const int64_t k = d.topk < d.T ? d.topk : d.T;
   for (int g = 0; g < ng; ++g)
@@ -252,6 +272,9 @@ int check_dims(const mla_dims* d) {
   if (d->B < 0 || d->T < 0 || d->H < 1 || d->T > MLA_MAX_T) return MLA_ERR_SHAPE;
   if (static_cast<int64_t>(d->B) * d->T > kMaxRows) return MLA_ERR_SHAPE;
   if (d->path != MLA_PATH_AUTO && d->path != MLA_PATH_BLOCK_DENSE && d->path != MLA_PATH_ABSORBED)
+    return MLA_ERR_UNSUPPORTED;
+  if (d->act != MLA_ACT_BF16 && d->act != MLA_ACT_E4M3_DYNAMIC) return MLA_ERR_UNSUPPORTED;
+  if (d->act == MLA_ACT_E4M3_DYNAMIC && (d->wdtype != MLA_W_E4M3_BLOCK128 || d->path == MLA_PATH_ABSORBED))
     return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
@@ -312,8 +335,20 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
     }
   }
   const bool dec = entry == MLA_ENTRY_DECODE;
-  if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
-  if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+  const bool act8 = d.act == MLA_ACT_E4M3_DYNAMIC;
+  if (act8) {
+    if (attend || entry == MLA_ENTRY_KV_UPPROJECT) {
+      w.lat8 = take(rows * kL);
+      w.lat8_s = take(rows * (kL / 128) * 4);
+    }
+    if (entry == MLA_ENTRY_PREFILL || entry == MLA_ENTRY_OUT_PROJECT) {
+      w.attn8 = take(rows * H * kDv);
+      w.attn8_s = take(rows * H * 4);
+    }
+  } else {
+    if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
+    if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+  }
   w.total = off;
   return w;
 }
@@ -386,6 +421,72 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
   if (M <= Gemm2WoNarrow::BM)
     return launch_gemm_pair<Gemm2WoNarrow>(ds->pairs_wo_narrow, ta, tb, tc, M, N, K, ds->err, 4, st);
   return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st);
+}
+
+// Dynamic e4m3 quantization of a bf16 [rows, cols] matrix: codes [rows, cols],
+// scales [cols / 128, rows].
+int launch_quant(const void* x, int rows, int cols, void* codes, float* scales, cudaStream_t st) {
+  const int64_t items = static_cast<int64_t>(rows) * (cols / 128);
+  const int64_t per_block = int64_t(2) * mla::kQuantWarps * mla::kQuantItemsPerHalfWarp;
+  const unsigned grid = static_cast<unsigned>((items + per_block - 1) / per_block);
+  if (grid == 0) return MLA_OK;
+  return timed_launch(8, st, [&] {
+    mla::quant_e4m3_1x128_kernel<<<grid, 32 * mla::kQuantWarps, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, cols, static_cast<uint8_t*>(codes), scales);
+  });
+}
+
+template <class Cfg>
+int launch_gemm8_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M,
+                      int N, int K, const mla::Gemm8Scales& sc, int* err, int cls, cudaStream_t st) {
+  const int tiles = ((M + Cfg::BM - 1) / Cfg::BM) * (N / Cfg::BN);
+  const int pairs = tiles < pairs_max ? tiles : pairs_max;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+  const int rc = timed_launch(
+      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_e4m3_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, sc, err); });
+  return le != cudaSuccess ? MLA_ERR_CUDA : rc;
+}
+
+// e4m3 up-projection: lat8 codes [M, 512] with scales [4, M] times the e4m3
+// W_kvb [H*256, 512] with block scales [2H, 4].
+int launch_gemm8_kvb(const DeviceState* ds, int M, int H, const void* lat8, const float* lat_s, const void* wkvb,
+                     const float* wkvb_s, void* kvh, bool v_f16, cudaStream_t st) {
+  const int N = H * (kDn + kDv), K = kL;
+  CUtensorMap ta, tb, tc;
+  if (!map_2d(&ta, lat8, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128) ||
+      !map_2d(&tb, wkvb, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 128, Gemm8Kvb::HN) ||
+      !map_2d(&tc, kvh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const mla::Gemm8Scales sc{lat_s, wkvb_s, 1, K / 128};
+  if (v_f16) return launch_gemm8_pair<Gemm8KvbAttn>(ds->pairs8_kvb, ta, tb, tc, M, N, K, sc, ds->err, 2, st);
+  return launch_gemm8_pair<Gemm8Kvb>(ds->pairs8_kvb, ta, tb, tc, M, N, K, sc, ds->err, 2, st);
+}
+
+// e4m3 output projection: attn8 codes [M, H*128] with scales [H, M] times
+// the e4m3 W_o [H*128, 7168] with block scales [H, 56].
+int launch_gemm8_wo(const DeviceState* ds, int M, int H, const void* attn8, const float* attn_s, const void* wo,
+                    const float* wo_s, void* out, cudaStream_t st) {
+  const int N = kD, K = H * kDv;
+  CUtensorMap ta, tb, tc;
+  if (!map_2d(&ta, attn8, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, 128) ||
+      !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, Gemm8Wo::HN, 128,
+              Gemm8Wo::HN == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map_2d(&tc, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32))
+    return MLA_ERR_CUDA;
+  const mla::Gemm8Scales sc{attn_s, wo_s, N / 128, 1};
+  return launch_gemm8_pair<Gemm8Wo>(ds->pairs8_wo, ta, tb, tc, M, N, K, sc, ds->err, 4, st);
 }
 
 int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks,
@@ -565,6 +666,14 @@ int begin_call(const mla_dims* dims, int entry, bool has_topk, void* ws, size_t 
 // it is stored as e4m3.
 int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* lat,
                   const void* W_kvb, const float* W_kvb_scale, void* kvh, bool v_f16, cudaStream_t st) {
+  if (d.act == MLA_ACT_E4M3_DYNAMIC) {
+    const int M = d.B * d.T;
+    void* lat8 = ws_at(ws, lay.lat8);
+    float* lat_s = reinterpret_cast<float*>(ws_at(ws, lay.lat8_s));
+    int rc = launch_quant(lat, M, kL, lat8, lat_s, st);
+    if (rc != MLA_OK) return rc;
+    return launch_gemm8_kvb(ds, M, d.H, lat8, lat_s, W_kvb, W_kvb_scale, kvh, v_f16, st);
+  }
   const void* wk = W_kvb;
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
     void* dq = ws_at(ws, lay.wkvb);
@@ -582,7 +691,8 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   const int ng = (nq + 3) / 4;
   const void* wk = W_kvb;
   int rc = MLA_OK;
-  if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+  const bool act8 = d.act == MLA_ACT_E4M3_DYNAMIC;  // every row block-dense (absorbed_first_group)
+  if (d.wdtype == MLA_W_E4M3_BLOCK128 && !act8) {
     void* dq = ws_at(ws, lay.wkvb);
     rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st);
     if (rc != MLA_OK) return rc;
@@ -591,7 +701,8 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   void* kvh = nullptr;
   if (lay.g_abs > 0) {  // up-projected keys, for the block-dense rows only
     kvh = ws_at(ws, lay.kvh);
-    rc = launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, /*v_f16=*/true, st);
+    rc = act8 ? run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, /*v_f16=*/true, st)
+              : launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, /*v_f16=*/true, st);
     if (rc != MLA_OK) return rc;
   }
   void* bitmap = nullptr;
@@ -632,6 +743,14 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
 
 int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* attn,
                     const void* W_o, const float* W_o_scale, void* out, cudaStream_t st) {
+  if (d.act == MLA_ACT_E4M3_DYNAMIC) {
+    const int M = d.B * d.T;
+    void* attn8 = ws_at(ws, lay.attn8);
+    float* attn_s = reinterpret_cast<float*>(ws_at(ws, lay.attn8_s));
+    int rc = launch_quant(attn, M, d.H * kDv, attn8, attn_s, st);
+    if (rc != MLA_OK) return rc;
+    return launch_gemm8_wo(ds, M, d.H, attn8, attn_s, W_o, W_o_scale, out, st);
+  }
   const void* wo = W_o;
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
     void* dq = ws_at(ws, lay.wo);
@@ -683,6 +802,7 @@ extern "C" {
 
 size_t mla_workspace_bytes(const mla_dims* dims, int entry, int has_topk) {
   if (check_dims(dims) != MLA_OK || entry < MLA_ENTRY_KV_UPPROJECT || entry > MLA_ENTRY_DECODE) return 0;
+  if (entry == MLA_ENTRY_DECODE && dims->act != MLA_ACT_BF16) return 0;
   return ws_layout(*dims, entry, has_topk != 0).total;
 }
 
@@ -782,10 +902,23 @@ int mla_decode(const mla_dims* dims, const void* q, const void* kv_latent, const
   if (!aligned16(q) || !aligned16(kv_latent) || !aligned16(k_pe) || !aligned16(W_kvb) || !aligned16(W_o) ||
       !aligned16(out) || !aligned16(W_kvb_scale) || !aligned16(W_o_scale) || !aligned16(topk_idx))
     return MLA_ERR_ALIGN;
+  if (dims->act != MLA_ACT_BF16) return MLA_ERR_UNSUPPORTED;
   rc = begin_call(dims, MLA_ENTRY_DECODE, topk_idx != nullptr, workspace, ws_bytes, &ds, &lay);
   if (rc != MLA_OK) return rc;
   return run_decode(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, W_o, W_o_scale, topk_idx,
                     scale, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_quantize_act(const void* x, int rows, int cols, void* codes, float* scales, mla_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 128 != 0) return MLA_ERR_SHAPE;
+  if (static_cast<int64_t>(rows) * cols >= (int64_t(1) << 40)) return MLA_ERR_SHAPE;
+  if (rows == 0) return MLA_OK;
+  if (!x || !codes || !scales) return MLA_ERR_NULL;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return MLA_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  const int rc = device_state(&ds);
+  if (rc != MLA_OK) return rc;
+  return launch_quant(x, rows, cols, codes, scales, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* mla_status_str(int status) {

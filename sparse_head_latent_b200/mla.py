@@ -20,10 +20,11 @@ _lib = None
 
 MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL, MLA_ENTRY_DECODE = 0, 1, 2, 3, 4
 MLA_W_BF16, MLA_W_E4M3_BLOCK128 = 0, 1
-MLA_PROFILE_CLASSES = 8
+MLA_PROFILE_CLASSES = 9
 MLA_PATH_AUTO, MLA_PATH_BLOCK_DENSE, MLA_PATH_ABSORBED = 0, 1, 2
+MLA_ACT_BF16, MLA_ACT_E4M3_DYNAMIC = 0, 1
 PROFILE_CLASS_NAMES = ("topk_prepass", "weight_dequant", "gemm_kvb", "attention", "gemm_wo", "row_lists",
-                       "gemm_absorb", "attention_absorbed")
+                       "gemm_absorb", "attention_absorbed", "act_quant")
 D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL = 128, 64, 128, 512, 7168
 
 
@@ -31,7 +32,7 @@ class MlaDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
                 ("d_nope", ctypes.c_int), ("d_rope", ctypes.c_int), ("d_v", ctypes.c_int),
                 ("d_latent", ctypes.c_int), ("d_model", ctypes.c_int),
-                ("topk", ctypes.c_int), ("wdtype", ctypes.c_int), ("path", ctypes.c_int)]
+                ("topk", ctypes.c_int), ("wdtype", ctypes.c_int), ("path", ctypes.c_int), ("act", ctypes.c_int)]
 
 
 class MlaError(RuntimeError):
@@ -54,6 +55,7 @@ SIGNATURES = {
                                   ctypes.c_float, _VP, _VP, _SZ, _VP]),
     "mla_attend_static": (ctypes.c_int, [ctypes.POINTER(MlaDims), _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_float,
                                          _VP, _VP]),
+    "mla_quantize_act": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP]),
     "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int)]),
     "mla_profile_begin": (ctypes.c_int, []),
@@ -106,9 +108,9 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_dims(B, T, H, topk=0, fp8=False, path=MLA_PATH_AUTO) -> MlaDims:
+def make_dims(B, T, H, topk=0, fp8=False, path=MLA_PATH_AUTO, act=MLA_ACT_BF16) -> MlaDims:
     return MlaDims(int(B), int(T), int(H), D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL, int(topk),
-                   MLA_W_E4M3_BLOCK128 if fp8 else MLA_W_BF16, int(path))
+                   MLA_W_E4M3_BLOCK128 if fp8 else MLA_W_BF16, int(path), int(act))
 
 
 def _wtype(w: torch.Tensor) -> bool:
@@ -130,11 +132,12 @@ def _workspace(dims, entry, has_topk, workspace, device):
     return workspace, workspace.numel() * workspace.element_size()
 
 
-def mla_kv_upproject(kv_latent, W_kvb, W_kvb_scale=None, kvh_out=None, workspace=None, stream=None):
+def mla_kv_upproject(kv_latent, W_kvb, W_kvb_scale=None, kvh_out=None, workspace=None, stream=None,
+                     act=MLA_ACT_BF16):
     """kv_latent bf16 [..., 512] -> kvh bf16 [rows, H*256]."""
     rows = kv_latent.numel() // D_LATENT
     H = W_kvb.shape[0] // (D_NOPE + D_V)
-    dims = make_dims(1, rows, H, 0, _wtype(W_kvb))
+    dims = make_dims(1, rows, H, 0, _wtype(W_kvb), act=act)
     if kvh_out is None:
         kvh_out = torch.empty(rows, H * (D_NOPE + D_V), dtype=torch.bfloat16, device=kv_latent.device)
     ws, nbytes = _workspace(dims, MLA_ENTRY_KV_UPPROJECT, False, workspace, kv_latent.device)
@@ -146,11 +149,11 @@ def mla_kv_upproject(kv_latent, W_kvb, W_kvb_scale=None, kvh_out=None, workspace
 
 
 def mla_attend(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale=192 ** -0.5,
-               attn_out=None, workspace=None, stream=None, path=MLA_PATH_AUTO):
+               attn_out=None, workspace=None, stream=None, path=MLA_PATH_AUTO, act=MLA_ACT_BF16):
     """q [B,T,H,192], kv_latent [B,T,512], k_pe [B,T,64] (bf16) -> attn bf16 [B,T,H,128]."""
     B, T, H, _ = q.shape
     topk = 0 if topk_idx is None else topk_idx.shape[-1]
-    dims = make_dims(B, T, H, topk, _wtype(W_kvb), path)
+    dims = make_dims(B, T, H, topk, _wtype(W_kvb), path, act)
     if topk_idx is not None and topk_idx.dtype != torch.int32:
         raise ValueError("topk_idx must be int32")
     if attn_out is None:
@@ -184,11 +187,11 @@ def mla_attend_static(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None
     return attn_out
 
 
-def mla_out_project(attn, W_o, W_o_scale=None, out=None, workspace=None, stream=None):
+def mla_out_project(attn, W_o, W_o_scale=None, out=None, workspace=None, stream=None, act=MLA_ACT_BF16):
     """attn bf16 [rows, H*128] (or [B,T,H,128]) -> out bf16 [rows, 7168]."""
     H = W_o.shape[0] // D_V
     rows = attn.numel() // (H * D_V)
-    dims = make_dims(1, rows, H, 0, _wtype(W_o))
+    dims = make_dims(1, rows, H, 0, _wtype(W_o), act=act)
     if out is None:
         out = torch.empty(rows, D_MODEL, dtype=torch.bfloat16, device=attn.device)
     ws, nbytes = _workspace(dims, MLA_ENTRY_OUT_PROJECT, False, workspace, attn.device)
@@ -199,7 +202,7 @@ def mla_out_project(attn, W_o, W_o_scale=None, out=None, workspace=None, stream=
 
 
 def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk_idx=None,
-                scale=192 ** -0.5, out=None, workspace=None, stream=None, path=MLA_PATH_AUTO):
+                scale=192 ** -0.5, out=None, workspace=None, stream=None, path=MLA_PATH_AUTO, act=MLA_ACT_BF16):
     """The whole attend block: -> out bf16 [B, T, 7168]."""
     B, T, H, _ = q.shape
     topk = 0 if topk_idx is None else topk_idx.shape[-1]
@@ -208,7 +211,7 @@ def mla_prefill(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None
         raise ValueError("W_kvb and W_o must use the same storage type")
     if topk_idx is not None and topk_idx.dtype != torch.int32:
         raise ValueError("topk_idx must be int32")
-    dims = make_dims(B, T, H, topk, fp8, path)
+    dims = make_dims(B, T, H, topk, fp8, path, act)
     if out is None:
         out = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=q.device)
     ws, nbytes = _workspace(dims, MLA_ENTRY_PREFILL, topk_idx is not None, workspace, q.device)
@@ -240,6 +243,21 @@ def mla_decode(q, kv_latent, k_pe, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None,
                                         _ptr(W_kvb_scale), _ptr(W_o), _ptr(W_o_scale), _ptr(topk_idx), float(scale),
                                         _ptr(out), _ptr(ws), nbytes, _stream(stream)))
     return out
+
+
+def mla_quantize_act(x, codes=None, scales=None, stream=None):
+    """Dynamic e4m3 quantization of x bf16 [rows, cols] (cols % 128 == 0) ->
+    (codes uint8 [rows, cols], scales float32 [cols // 128, rows]), s = amax / 448 per group."""
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    rows, cols = x.reshape(-1, x.shape[-1]).shape
+    if codes is None:
+        codes = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(cols // 128 if cols % 128 == 0 else 0, rows, dtype=torch.float32, device=x.device)
+    _check("mla_quantize_act", load_library().mla_quantize_act(_ptr(x), rows, cols, _ptr(codes), _ptr(scales),
+                                                               _stream(stream)))
+    return codes, scales
 
 
 def mla_device_status(stream=None) -> int:
@@ -274,7 +292,7 @@ class PrefillPipeline:
     _INPUTS = ("q", "kv_latent", "k_pe", "topk_idx")
 
     def __init__(self, B, T, H, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk=None,
-                 scale=192 ** -0.5, device=None):
+                 scale=192 ** -0.5, device=None, act=MLA_ACT_BF16):
         dev = torch.device(device) if device is not None else W_o.device
         self.dev, self.scale = dev, float(scale)
         self.w = dict(W_kvb=W_kvb, W_o=W_o, W_kvb_scale=W_kvb_scale, W_o_scale=W_o_scale)
@@ -285,7 +303,8 @@ class PrefillPipeline:
         self.slots = [{k: torch.empty(s, dtype=d, device=dev) for k, (s, d) in shapes.items()} for _ in range(2)]
         for sl in self.slots:
             sl["out"] = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=dev)
-        dims = make_dims(B, T, H, 0 if topk is None else topk, _wtype(W_kvb))
+        self.act = int(act)
+        dims = make_dims(B, T, H, 0 if topk is None else topk, _wtype(W_kvb), act=self.act)
         self.ws = torch.empty(max(1, mla_workspace_bytes(dims, MLA_ENTRY_PREFILL, topk is not None)),
                               dtype=torch.uint8, device=dev)
         self.h2d, self.comp, self.d2h = (torch.cuda.Stream(dev) for _ in range(3))
@@ -311,7 +330,7 @@ class PrefillPipeline:
             self.comp.wait_event(self.ev_out[k])  # the previous output of this slot has been copied out
         mla_prefill(sl["q"], sl["kv_latent"], sl["k_pe"], self.w["W_kvb"], self.w["W_o"], self.w["W_kvb_scale"],
                     self.w["W_o_scale"], topk_idx=sl.get("topk_idx"), scale=self.scale, out=sl["out"],
-                    workspace=self.ws, stream=self.comp)
+                    workspace=self.ws, stream=self.comp, act=self.act)
         self.ev_done[k].record(self.comp)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.ev_done[k])

@@ -83,6 +83,48 @@ def test_workspace_sizes_absorbed_path(lib):
     assert mla.mla_workspace_bytes(_dims(path=3), mla.MLA_ENTRY_ATTEND, True) == 0
 
 
+def test_workspace_sizes_e4m3_activations(lib):
+    # Quantized latent (1 byte per element + one fp32 scale per 128) and
+    # quantized attention rows; no dequantized weight copies.
+    T, H = 256, 4
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    d = _dims(wdtype=1, act=mla.MLA_ACT_E4M3_DYNAMIC)
+    lat8 = up(T * 512) + up(T * 4 * 4)
+    attn8 = up(T * H * 128) + up(T * H * 4)
+    kvh = up(T * H * 256 * 2)
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_KV_UPPROJECT, False) == lat8
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_OUT_PROJECT, False) == attn8
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, False) == kvh + lat8
+    # AUTO with top-k stays block-dense (the absorbed rows have no quantized form)
+    nq = 2
+    sel = up(nq * (nq + 1) // 2 * 128 * 16) + up(nq * (nq + 1) * 4)
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_ATTEND, True) == kvh + sel + lat8
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_PREFILL, True) == kvh + up(T * H * 128 * 2) + sel + lat8 + attn8
+    # unsupported combinations report no workspace
+    assert mla.mla_workspace_bytes(_dims(act=1), mla.MLA_ENTRY_ATTEND, False) == 0          # bf16 weights
+    assert mla.mla_workspace_bytes(_dims(wdtype=1, act=1, path=mla.MLA_PATH_ABSORBED),
+                                   mla.MLA_ENTRY_ATTEND, True) == 0
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_DECODE, True) == 0
+    assert mla.mla_workspace_bytes(_dims(wdtype=1, act=2), mla.MLA_ENTRY_ATTEND, False) == 0
+
+
+def test_e4m3_activation_host_checks(lib):
+    sc = 16
+    assert _attend(lib, _dims(act=1)) == 3                                     # needs e4m3 weights
+    assert _attend(lib, _dims(wdtype=1, act=1, path=mla.MLA_PATH_ABSORBED), {"sc": sc, "tk": 16}) == 3
+    assert _attend(lib, _dims(wdtype=1, act=7), {"sc": sc}) == 3
+    assert _attend(lib, _dims(wdtype=1, act=1), {"sc": sc}) == 4               # workspace missing
+    d = _dims(wdtype=1, act=1)
+    assert lib.mla_decode(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 16, None, ctypes.c_float(0.1), 16, 16, 1 << 30,
+                          None) == 3
+    # the stand-alone quantizer validates before touching the device
+    assert lib.mla_quantize_act(16, 4, 100, 16, 16, None) == 2                  # cols not a multiple of 128
+    assert lib.mla_quantize_act(16, -1, 128, 16, 16, None) == 2
+    assert lib.mla_quantize_act(None, 4, 128, 16, 16, None) == 1
+    assert lib.mla_quantize_act(24, 4, 128, 16, 16, None) == 6
+    assert lib.mla_quantize_act(None, 0, 128, None, None, None) == 0           # nothing to do
+
+
 def _attend(lib, d, ptrs=None, scale=0.07, ws=None, nbytes=0):
     p = dict(q=16, lat=16, kpe=16, wk=16, sc=None, tk=None, out=16)
     p.update(ptrs or {})

@@ -36,7 +36,8 @@ MUTANTS = [
                              "for (int c = 0; c < mark[t]; ++c) sel[n].push_back(t);")]),
     ("out_of_range_wraps", [("if (t >= 0 && t < T && t <= s) mark[t] = 1;",
                              "if (t <= s) mark[((t % T) + T) % T] = 1;")]),
-    ("wo_row_reversed", [("const double ak = a[k];", "const double ak = a[K - 1 - k];")]),
+    ("wo_row_reversed", [("const double ak = rows_in[static_cast<size_t>(n) * K + k];",
+                          "const double ak = rows_in[static_cast<size_t>(n) * K + K - 1 - k];")]),
     ("e4m3_bias", [("ex - 7);", "ex - 8);")]),
     ("e4m3_subnormal_exponent", [("static_cast<double>(man) / 8.0, -6);", "static_cast<double>(man) / 8.0, -7);")]),
     ("bf16_shift", [("static_cast<uint32_t>(bits) << 16;", "static_cast<uint32_t>(bits) << 15;")]),
