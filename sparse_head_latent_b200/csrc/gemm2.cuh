@@ -39,6 +39,7 @@ struct Gemm2Cfg {
   static constexpr bool B_MN_MAJOR = B_MN_MAJOR_;
   static constexpr bool V_F16 = V_F16_;
   static constexpr int STAGES = 6;
+  static constexpr int GROUP_M = 8;             // row tiles per group of the tile order (grouped_tile)
   static constexpr int A_BYTES = HM * BK * 2;   // 16 KB
   static constexpr int B_BYTES = HN * BK * 2;   // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -134,7 +135,9 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int it = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % num_m, nt = (tile / num_m) % num_n, bi = tile / (num_m * num_n);
+        const int bi = tile / (num_m * num_n);
+        int mt, nt;
+        grouped_tile(tile - bi * num_m * num_n, num_m, num_n, Cfg::GROUP_M, mt, nt);
         const int arow = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM;
         const int bcol = nt * Cfg::BN + static_cast<int>(rank) * Cfg::HN;
         const int acol0 = bt.a_col0 + bi * bt.a_col_step;
@@ -210,7 +213,9 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* bufs = epi + (warp - 2) * 2 * Cfg::EPI_BUF;
     int t = 0, nbuf = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
-      const int mt = tile % num_m, nt = (tile / num_m) % num_n, bi = tile / (num_m * num_n);
+      const int bi = tile / (num_m * num_n);
+      int mt, nt;
+      grouped_tile(tile - bi * num_m * num_n, num_m, num_n, Cfg::GROUP_M, mt, nt);
       const int a = t & 1;
       const uint32_t aph = (t >> 1) & 1;
       if (!warp_wait(accf0 + 8 * a, aph, ab, kErrWaitMma)) break;

@@ -56,6 +56,7 @@ struct Gemm8Cfg {
   static constexpr int B_BYTES = HN * BK;   // 8 or 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN_ == 128 ? 6 : 5;
+  static constexpr int GROUP_M = 8;          // row tiles per group of the tile order (grouped_tile)
   static constexpr int ACC_BUFS = 512 / BN_;  // BN-column partial buffers
   static constexpr int PROMO_WARPS = 8;
   static constexpr int CW = BN_ / 2;         // columns per promotion warp
@@ -140,7 +141,8 @@ gemm_e4m3_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int it = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % num_m, nt = tile / num_m;
+        int mt, nt;
+        grouped_tile(tile, num_m, num_n, Cfg::GROUP_M, mt, nt);
         const int arow = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM;
         const int bcol = nt * Cfg::BN + static_cast<int>(rank) * Cfg::HN;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
@@ -219,7 +221,8 @@ gemm_e4m3_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     int pc = 0, nbuf = 0;
     bool ok = true;
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-      const int mt = tile % num_m, nt = tile / num_m;
+      int mt, nt;
+      grouped_tile(tile, num_m, num_n, Cfg::GROUP_M, mt, nt);
       const int row0 = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM + q * 32;
       const int row = row0 + static_cast<int>(lane);
       const bool live = row < M;

@@ -33,8 +33,8 @@ using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as 
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
 using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
-using Gemm8Kvb = mla::Gemm8Cfg<false>;         // e4m3 latent x e4m3 W_kvb^T
-using Gemm8KvbAttn = mla::Gemm8Cfg<false, true>;  // same, v tiles written as f16 for the attention
+using Gemm8Kvb = mla::Gemm8Cfg<false>;              // e4m3 latent x e4m3 W_kvb^T
+using Gemm8KvbAttn = mla::Gemm8Cfg<false, true>;    // same, v tiles written as f16 for the attention
 using Gemm8Wo = mla::Gemm8Cfg<true>;           // e4m3 attn x e4m3 W_o (B stored [K, N])
 
 // ------------------------------------------------------------------ device state

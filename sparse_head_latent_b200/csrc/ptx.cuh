@@ -450,6 +450,24 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask
       : "memory");
 }
 
+// ------------------------------------------------------------------ tile order
+
+// Persistent GEMMs walk their output tiles in groups of `group_m` row tiles:
+// within a group, row tiles vary fastest and column tiles follow, so the
+// resident CTAs share a band of A rows (group_m x 256 rows, reused across
+// every column tile) and each B column block is fetched once per group. A
+// plain row-fastest order streams all of A once per column tile, which for
+// an A larger than L2 multiplies its DRAM reads by the column-tile count.
+__device__ __forceinline__ void grouped_tile(int tile, int num_m, int num_n, int group_m, int& mt, int& nt) {
+  const int per_group = group_m * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * group_m;
+  const int gm = num_m - first_m < group_m ? num_m - first_m : group_m;
+  const int within = tile - g * per_group;
+  mt = first_m + within % gm;
+  nt = within / gm;
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor (tcgen05 form): start address, leading and
