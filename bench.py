@@ -60,6 +60,9 @@ def parse_args(argv=None):
     p.add_argument("--T", type=int, default=None, help="override the workload's sequence length")
     p.add_argument("--H", type=int, default=None, help="override the workload's head count")
     p.add_argument("--topk", type=int, default=None, help="override the workload's top-k")
+    p.add_argument("--parallel", choices=["sequences", "heads"], default="sequences",
+                   help="N > 1: independent sequences per rank (weak scaling) or one problem with its heads "
+                        "split over the ranks and the partial outputs all-reduced (strong scaling)")
     p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
                    help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
     return p.parse_args(argv)
@@ -423,6 +426,114 @@ def run_ours(args, rank, world, local):
     return result
 
 
+def run_heads(args, rank, world, local):
+    """One problem of the workload with its heads split over the ranks
+    (sparse_head_latent_b200.tp.HeadShardedPrefill): per step every rank runs
+    its heads' attention and W_o rows and the partial outputs are all-reduced
+    in row chunks overlapped with the projection. `value` is the problem's
+    algorithmic FLOPs over the max-over-ranks step time (strong scaling)."""
+    import sparse_head_latent_b200 as mla
+    from sparse_head_latent_b200.tp import HeadShardedPrefill
+
+    name, x = workload(args)
+    wm = work_model(x)
+    dev = torch.device("cuda", local)
+    act = mla.MLA_ACT_E4M3_DYNAMIC if args.act == "e4m3" else mla.MLA_ACT_BF16
+    tk = x.topk_idx.shape[-1] if x.topk_idx is not None else None
+    g = {k: v.to(dev) for k, v in x.tensors().items() if k not in ("q",)}
+    tp = HeadShardedPrefill(x.B, x.T, x.H, g["W_kvb"], g["W_o"], g.get("W_kvb_scale"), g.get("W_o_scale"), topk=tk,
+                            scale=x.scale, act=act, device=dev)
+    q_local = x.q[:, :, tp.h0:tp.h1].contiguous().to(dev)
+    out = torch.empty(x.B, x.T, 7168, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tp(q_local, g["kv_latent"], g["k_pe"], g.get("topk_idx"), out=out)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local).start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mla.mla_profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = mla.mla_profile_end()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    # End to end: the rank's inputs from pinned host memory and the output back, every step.
+    host = {"q": q_local.cpu().pin_memory(), "kv_latent": g["kv_latent"].cpu().pin_memory(),
+            "k_pe": g["k_pe"].cpu().pin_memory()}
+    if g.get("topk_idx") is not None:
+        host["topk_idx"] = g["topk_idx"].cpu().pin_memory()
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = args.e2e_steps or args.steps
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        tp(dev_in["q"], dev_in["kv_latent"], dev_in["k_pe"], dev_in.get("topk_idx"), out=out)
+        host_out.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(world)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world)
+    clocks.stop()
+    if mla.mla_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    tflops = wm["flops"] / (ms * 1e-3) / 1e12
+    kflops = {"gemm_kvb": wm["flops_kvb"] / world, "attention": wm["flops_attn"] / world,
+              "gemm_wo": wm["flops_wo"] / world}
+    # Work per step of each kernel class on this rank (W_o runs once per row
+    # chunk, so rates are per step, not per launch).
+    per_kernel = {}
+    for kname, (tot_ms, n) in prof.items():
+        if n:
+            per_kernel[kname] = {"launches": n, "avg_ms": round(tot_ms / n, 5)}
+            if kname in kflops:
+                per_kernel[kname]["tflops"] = round(kflops[kname] / (tot_ms / args.steps * 1e-3) / 1e12, 1)
+    dom = max((k for k in per_kernel if k in kflops), key=lambda k: prof[k][0])
+    achieved = kflops[dom] / (prof[dom][0] / args.steps * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {
+        "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "e4m3 x e4m3 projections, bf16 attention" if act else "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the workload; no checkpoint)",
+        "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
+                   "weights": "e4m3 block-128" if x.fp8 else "bf16",
+                   "activations": "e4m3 dynamic 1x128" if act else "bf16",
+                   "parallelism": f"heads split over {world} ranks, partial outputs all-reduced (NCCL)",
+                   "l2": "no flush: every step reads more than the 126 MB L2"},
+        "queries_per_s": round(x.B * x.T / (ms * 1e-3), 1),
+        "per_kernel": per_kernel,
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst), MEASURED_PEAKS.json"},
+        "e2e": {"value": round(wm["flops"] / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": int(sum(n for _, n in prof.values())),
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+
+
 # ------------------------------------------------------------------ reference arm (CPU oracle)
 
 def run_decode(args, local):
@@ -537,7 +648,12 @@ def main(argv=None):
     else:
         rank, world, local = dist_setup()
         try:
-            res = run_decode(args, local) if args.mode == "decode" else run_ours(args, rank, world, local)
+            if args.mode == "decode":
+                res = run_decode(args, local)
+            elif args.parallel == "heads":
+                res = run_heads(args, rank, world, local)
+            else:
+                res = run_ours(args, rank, world, local)
         finally:
             if world > 1:
                 import torch.distributed as dist
