@@ -55,6 +55,11 @@ struct AttnParams {
   const uint4* bitmap;          // selection bitmap, NULL = causal mask only
   const int32_t* blocks;        // active key blocks per tile group (with bitmap)
   __nv_bfloat16* attn;          // [B, T, H, 128]
+  // When set, the output is written as dynamic e4m3 activations instead of
+  // bf16 (the input of an e4m3 x e4m3 output projection): each (row, head)
+  // is one 128-channel group; codes [B*T, H*128], scales [H, B*T].
+  uint8_t* attn8;
+  float* attn8_s;
   int* err;
 };
 
@@ -432,6 +437,39 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           if (ok) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            if (p.attn8 != nullptr) {
+              // e4m3 output: the row's 128 values, rounded to bf16 as the
+              // bf16 path stores them, quantized as one group (s = amax / 448,
+              // code = e4m3(v / s), divisions rounded to nearest even).
+              uint32_t a[128];
+              tmem_ld128(tO, a);
+              float amax = 0.f;
+#pragma unroll
+              for (int i = 0; i < 128; ++i) {
+                const float v = __bfloat162float(__float2bfloat16_rn(__uint_as_float(a[i]) * inv));
+                a[i] = __float_as_uint(v);
+                amax = fmaxf(amax, fabsf(v));
+              }
+              const float sc = __fdiv_rn(amax, 448.0f);
+              if (s < p.T) {
+                const int64_t row = static_cast<int64_t>(b) * p.T + s;
+                uint4* d4 = reinterpret_cast<uint4*>(p.attn8 + (row * p.H + h) * 128);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  uint32_t w[4];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const float* v = reinterpret_cast<const float*>(a) + 16 * i + 4 * k;
+                    w[k] = sc == 0.f ? 0u
+                                     : (static_cast<uint32_t>(pack_e4m3x2(__fdiv_rn(v[0], sc), __fdiv_rn(v[1], sc))) |
+                                        (static_cast<uint32_t>(pack_e4m3x2(__fdiv_rn(v[2], sc), __fdiv_rn(v[3], sc)))
+                                         << 16));
+                  }
+                  d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                p.attn8_s[static_cast<int64_t>(h) * p.B * p.T + row] = sc;
+              }
+            } else {
 #pragma unroll 1
             for (int c0 = 0; c0 < 128; c0 += 64) {
               uint32_t a0[32], a1[32];
@@ -451,10 +489,18 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
               }
             }
+            }
           }
-        } else if (s < p.T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-          for (int i = 0; i < 16; ++i) d4[i] = make_uint4(0, 0, 0, 0);  // no surviving key
+        } else if (s < p.T) {  // no surviving key
+          if (p.attn8 != nullptr) {
+            const int64_t row = static_cast<int64_t>(b) * p.T + s;
+            uint4* d4 = reinterpret_cast<uint4*>(p.attn8 + (row * p.H + h) * 128);
+            for (int i = 0; i < 8; ++i) d4[i] = make_uint4(0, 0, 0, 0);
+            p.attn8_s[static_cast<int64_t>(h) * p.B * p.T + row] = 0.f;
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            for (int i = 0; i < 16; ++i) d4[i] = make_uint4(0, 0, 0, 0);
+          }
         }
       }
     }

@@ -295,7 +295,9 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
   if (attend) {
     w.g_abs = absorbed_first_group(d, has_topk);
     if (w.g_abs > 0) w.kvh = take(rows * H * (kDn + kDv) * 2);  // block-dense rows only
-    if (entry == MLA_ENTRY_PREFILL) w.attn = take(rows * H * kDv * 2);
+    // The whole block keeps the attention rows in the workspace (as e4m3
+    // codes + scales when the activations are quantized, see below).
+    if (entry == MLA_ENTRY_PREFILL && d.act != MLA_ACT_E4M3_DYNAMIC) w.attn = take(rows * H * kDv * 2);
     if (has_topk) {
       w.bitmap = take(static_cast<size_t>(d.B) * (nq * (nq + 1) / 2) * 128 * 16);
       w.blocks = take(static_cast<size_t>(d.B) * ((nq + 3) / 4) * (nq + 2) * 4);
@@ -509,9 +511,11 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
 }
 
 // Block-dense attention for tile groups [0, ngroups_run).
+// attn8 / attn8_s set: the output is written as e4m3 codes + scales (the
+// input of the e4m3 output projection) instead of bf16.
 int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, const void* kvh, const void* k_pe,
                      const void* bitmap, const void* blocks, float scale, void* attn, int ngroups_run,
-                     cudaStream_t st) {
+                     cudaStream_t st, void* attn8 = nullptr, float* attn8_s = nullptr) {
   // Q tiles and V blocks are 128 rows; each CTA of a pair loads 64 keys of K.
   CUtensorMap tq, tk, tv, tpe;
   const uint64_t kv_inner = static_cast<uint64_t>(d.H) * (kDn + kDv);
@@ -539,6 +543,8 @@ int launch_attention(const DeviceState* ds, const mla_dims& d, const void* q, co
   p.bitmap = static_cast<const uint4*>(bitmap);
   p.blocks = static_cast<const int32_t*>(blocks);
   p.attn = static_cast<__nv_bfloat16*>(attn);
+  p.attn8 = static_cast<uint8_t*>(attn8);
+  p.attn8_s = attn8_s;
   p.err = ds->err;
   const int64_t pairs = static_cast<int64_t>(d.B) * p.ngroups * d.H;
   cudaLaunchConfig_t cfg = {};
@@ -686,7 +692,8 @@ int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay,
 
 int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, void* ws, const void* q,
                const void* lat, const void* k_pe, const void* W_kvb, const float* W_kvb_scale,
-               const int32_t* topk_idx, float scale, void* attn, cudaStream_t st) {
+               const int32_t* topk_idx, float scale, void* attn, cudaStream_t st, void* attn8 = nullptr,
+               float* attn8_s = nullptr) {
   const int nq = (d.T + 127) / 128;
   const int ng = (nq + 3) / 4;
   const void* wk = W_kvb;
@@ -714,7 +721,7 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
     if (rc != MLA_OK) return rc;
   }
   if (lay.g_abs > 0) {
-    rc = launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, lay.g_abs, st);
+    rc = launch_attention(ds, d, q, kvh, k_pe, bitmap, blocks, scale, attn, lay.g_abs, st, attn8, attn8_s);
     if (rc != MLA_OK) return rc;
   }
   if (lay.g_abs >= ng) return MLA_OK;
@@ -880,6 +887,16 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent, cons
   if (rc != MLA_OK) return rc;
   if (static_cast<int64_t>(dims->B) * dims->T == 0) return MLA_OK;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->act == MLA_ACT_E4M3_DYNAMIC) {
+    // The attention kernel writes its output already quantized (every row
+    // is block-dense with e4m3 activations), so W_o reads the codes directly.
+    void* attn8 = ws_at(workspace, lay.attn8);
+    float* attn8_s = reinterpret_cast<float*>(ws_at(workspace, lay.attn8_s));
+    rc = run_attend(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, nullptr, st,
+                    attn8, attn8_s);
+    if (rc != MLA_OK) return rc;
+    return launch_gemm8_wo(ds, dims->B * dims->T, dims->H, attn8, attn8_s, W_o, W_o_scale, out, st);
+  }
   void* attn = ws_at(workspace, lay.attn);
   rc = run_attend(ds, *dims, lay, workspace, q, kv_latent, k_pe, W_kvb, W_kvb_scale, topk_idx, scale, attn, st);
   if (rc != MLA_OK) return rc;
