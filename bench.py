@@ -587,6 +587,28 @@ def run_decode(args, local):
     if mla.mla_device_status(stream) != 0:
         raise RuntimeError("device error in the timed region")
     ms = e0.elapsed_time(e1) / args.steps
+    # End to end: every step copies its new inputs from pinned host memory --
+    # the queries, the selections and the new position's latent and rope rows
+    # (the cache itself stays resident) -- replays the step and copies the
+    # output back.
+    h_q, h_tk = g["q"].cpu().pin_memory(), g["topk_idx"].cpu().pin_memory()
+    h_lat, h_pe = g["kv_latent"][:, T - 1].cpu().pin_memory(), g["k_pe"][:, T - 1].cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_tk, h_lat, h_pe))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = args.e2e_steps or args.steps
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        g["q"].copy_(h_q, non_blocking=True)
+        g["topk_idx"].copy_(h_tk, non_blocking=True)
+        g["kv_latent"][:, T - 1].copy_(h_lat, non_blocking=True)
+        g["k_pe"][:, T - 1].copy_(h_pe, non_blocking=True)
+        graph.replay()
+        h_out.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
     del graph
     sel = min(k, T)
     compulsory = (H * 256 * 512 * 2 + H * 128 * 7168 * 2        # W_kvb, W_o
@@ -611,6 +633,8 @@ def run_decode(args, local):
         "per_kernel": per, "per_kernel_source": "eager profiled run of the same steps",
         "timing": "CUDA graph replay of the whole decode step",
         "gpu_launches": sum(c for _, c in prof.values()),
+        "e2e": {"value": round(B / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "clocks": clocks.summary(t_wall0, t_wall1),
     }
 
