@@ -61,3 +61,54 @@ def test_full_size_sampled_rows(name):
     assert_close(attn[torch.tensor(flat, device=attn.device)].float().cpu().numpy(), ref_attn,
                  f"{name} attn rows")
     assert np.isfinite(out.float().cpu().numpy()).all()
+
+
+def test_full_size_e4m3_activations_sampled_rows():
+    # The batched FP8 workload with dynamic e4m3 activations (the attention
+    # output is quantized in the attention kernel's epilogue). The whole block
+    # is held to the tolerance derived for the e4m3 path (code flips of the
+    # re-quantized attention rows, see test_gpu_act8) and must be closer to
+    # the quantized oracle than to the bf16-activation one.
+    from tests.test_gpu_act8 import BLOCK_MAX_ABS, BLOCK_REL_L2
+    x = synth.make_inputs(4)
+    g = {k: v.cuda() for k, v in x.tensors().items()}
+    act = mla.MLA_ACT_E4M3_DYNAMIC
+    out = mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g["W_kvb_scale"], g["W_o_scale"],
+                          topk_idx=g["topk_idx"], scale=x.scale, act=act)
+    attn = mla.mla_attend(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_kvb_scale"], topk_idx=g["topk_idx"],
+                          scale=x.scale, act=act)
+    assert mla.mla_device_status() == 0
+    del g
+    flat = [0 * x.T + 5, 7 * x.T + 511, 15 * x.T + 1023]
+    ref_attn, ref_q = oracle.prefill_rows(x, flat, act_e4m3=True)
+    _, ref_b = oracle.prefill_rows(x, flat)
+    got_attn = attn.view(-1, x.H, 128)[torch.tensor(flat, device=attn.device)].float().cpu().numpy()
+    assert_close(got_attn, ref_attn, "e4m3 act attn rows")
+    got = out.view(-1, 7168)[torch.tensor(flat, device=out.device)].float().cpu().numpy()
+    d_q = float(np.linalg.norm(got - ref_q) / np.linalg.norm(ref_q))
+    d_b = float(np.linalg.norm(got - ref_b) / np.linalg.norm(ref_b))
+    assert d_q <= BLOCK_REL_L2 and float(np.abs(got - ref_q).max()) <= BLOCK_MAX_ABS, d_q
+    assert d_q < 0.6 * d_b, (d_q, d_b)
+
+
+def test_full_size_decode_sampled_sequence():
+    # The decode workload of the benchmark (64 sequences, 32768-position
+    # caches, 128 heads, top-k 2048); one sequence's output is checked against
+    # the oracle's prefill row s = T - 1 of that sequence (its queries at the
+    # other positions are never read).
+    B, T, H, k = 64, 32768, 128, 2048
+    d = synth.make_decode_inputs(B, T, H, k, seed=11)
+    g = {n: v.cuda() for n, v in d.tensors().items()}
+    out = mla.mla_decode(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], topk_idx=g["topk_idx"],
+                         scale=d.scale)
+    assert mla.mla_device_status() == 0
+    b = 37
+    q = torch.zeros(1, T, H, 192, dtype=torch.bfloat16)
+    q[0, T - 1] = d.q[b]
+    tk = torch.zeros(1, T, k, dtype=torch.int32)
+    tk[0, T - 1] = d.topk_idx[b]
+    one = synth.MlaInputs(B=1, T=T, H=H, topk=k, fp8=False, scale=d.scale, q=q, kv_latent=d.kv_latent[b:b + 1],
+                          k_pe=d.k_pe[b:b + 1], W_kvb=d.W_kvb, W_kvb_scale=None, W_o=d.W_o, W_o_scale=None,
+                          topk_idx=tk)
+    _, ref = oracle.prefill_rows(one, [T - 1])
+    assert_close(out[b:b + 1].float().cpu().numpy(), ref, "decode sequence 37")
