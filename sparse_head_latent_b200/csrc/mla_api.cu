@@ -18,6 +18,7 @@
 #include "dequant.cuh"
 #include "gemm2.cuh"
 #include "gemm8.cuh"
+#include "gemm_m64.cuh"
 #include "prepass.cuh"
 #include "quant.cuh"
 #include "ptx.cuh"
@@ -33,6 +34,8 @@ using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as 
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
 using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
+using GemmM64 = mla::GemmM64Cfg<64>;     // decode's output projection, M <= 64
+using GemmM128 = mla::GemmM64Cfg<128>;   // and 64 < M <= 256 (128-row tiles)
 using Gemm8Kvb = mla::Gemm8Cfg<false>;              // e4m3 latent x e4m3 W_kvb^T
 using Gemm8KvbAttn = mla::Gemm8Cfg<false, true>;    // same, v tiles written as f16 for the attention
 using Gemm8Wo = mla::Gemm8Cfg<true>;           // e4m3 attn x e4m3 W_o (B stored [K, N])
@@ -125,6 +128,10 @@ int device_state(DeviceState** out) {
         st.pairs8_wo = max_pairs(mla::gemm_e4m3_tc2_kernel<Gemm8Wo>, Gemm8Wo::SMEM_BYTES, Gemm8Wo::THREADS);
         ok = st.pairs8_kvb > 0 && st.pairs8_wo > 0;
       }
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      GemmM64::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM128::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AbsSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -230,6 +237,8 @@ struct WsLayout {
   size_t lat8 = kNone, lat8_s = kNone;    // e4m3 activations: quantized latent and its scales
   size_t attn8 = kNone, attn8_s = kNone;  // e4m3 activations: quantized attention rows and scales
   int parts = 1;                          // decode: CTAs per (sequence, 64-head group)
+  int wo_splits = 1;                      // decode: K ranges of the output projection
+  size_t wo_part = kNone;                 // decode: their fp32 partial outputs [wo_splits, B, 7168]
   int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
   int abs_chunk = 0;   // absorbed rows processed per pass
   int kpad = 0;        // pitch of the per-row key lists
@@ -334,6 +343,12 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
     if (w.parts > 1) {
       w.part_ml = take(B * w.parts * H * 8);
       w.part_o = take(B * w.parts * H * kL * 2);
+    }
+    // The output projection of up to 256 rows runs as a split-K GEMM with
+    // M = 64 tiles: K = 128 H is cut into ranges of whole 64-deep blocks.
+    if (d.B <= 256) {
+      w.wo_splits = (2 * d.H) % 8 == 0 ? 8 : (2 * d.H) % 4 == 0 ? 4 : 2;
+      w.wo_part = take(static_cast<size_t>(w.wo_splits) * B * kD * 4);
     }
   }
   const bool dec = entry == MLA_ENTRY_DECODE;
@@ -489,6 +504,35 @@ int launch_gemm8_wo(const DeviceState* ds, int M, int H, const void* attn8, cons
     return MLA_ERR_CUDA;
   const mla::Gemm8Scales sc{attn_s, wo_s, N / 128, 1};
   return launch_gemm8_pair<Gemm8Wo>(ds->pairs8_wo, ta, tb, tc, M, N, K, sc, ds->err, 4, st);
+}
+
+// Output projection of M <= 256 rows as a split-K GEMM (M = 64 UMMA tiles):
+// fp32 partial outputs per K range into `part`, then summed into `out`.
+int launch_gemm_wo_m64(const DeviceState* ds, int M, int H, const void* attn, const void* wo, float* part,
+                       int splits, void* out, cudaStream_t st) {
+  const int N = kD, K = H * kDv;
+  if ((K / splits) % GemmM64::BK != 0) return MLA_ERR_SHAPE;
+  const int bm = M <= 64 ? 64 : 128;
+  CUtensorMap ta, tb;
+  if (!map_2d(&ta, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, bm) ||
+      !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64))
+    return MLA_ERR_CUDA;
+  const int items = ((M + bm - 1) / bm) * (N / GemmM64::BN) * splits;
+  const int grid = items < ds->sms ? items : ds->sms;
+  int rc = timed_launch(4, st, [&] {
+    if (bm == 64)
+      mla::gemm_m64_splitk_kernel<GemmM64><<<grid, GemmM64::THREADS, GemmM64::SMEM_BYTES, st>>>(
+          ta, tb, M, N, K, splits, part, ds->err);
+    else
+      mla::gemm_m64_splitk_kernel<GemmM128><<<grid, GemmM128::THREADS, GemmM128::SMEM_BYTES, st>>>(
+          ta, tb, M, N, K, splits, part, ds->err);
+  });
+  if (rc != MLA_OK) return rc;
+  const int64_t quads = static_cast<int64_t>(M) * N / 4;
+  return timed_launch(4, st, [&] {
+    mla::sum_splits_kernel<<<static_cast<unsigned>((quads + 255) / 256), 256, 0, st>>>(
+        part, M, N, splits, static_cast<__nv_bfloat16*>(out));
+  });
 }
 
 int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk, void* bitmap, void* blocks,
@@ -798,6 +842,9 @@ int run_decode(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
     if ((rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st)) != MLA_OK) return rc;
     wo = dq;
   }
+  if (lay.wo_splits > 1)
+    return launch_gemm_wo_m64(ds, d.B, d.H, attn, wo, reinterpret_cast<float*>(ws_at(ws, lay.wo_part)),
+                              lay.wo_splits, out, st);
   return launch_gemm_wo(ds, d.B, d.H, attn, wo, out, st);
 }
 
