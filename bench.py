@@ -40,7 +40,8 @@ import synth  # noqa: E402
 METRIC = "sparse MLA prefill TFLOP/s and queries/s (T=4096,H=128,top-k 2048); % of bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "quant.cuh", "attn.cuh", "attn_abs.cuh", "prepass.cuh",
+KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "gemm_m64.cuh", "quant.cuh", "attn.cuh", "attn_abs.cuh",
+                  "prepass.cuh",
                   "dequant.cuh", "mla_api.cu")
 
 

@@ -549,7 +549,7 @@ int launch_prepass(const DeviceState* ds, const mla_dims& d, const int32_t* topk
   if (rc != MLA_OK) return rc;
   dim3 grid((nq + 3) / 4, d.B);
   return timed_launch(0, st, [&] {
-    mla::topk_block_list_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4*>(bitmap), nq,
+    mla::topk_block_list_kernel<<<grid, 32 * mla::kBlockListWarps, 0, st>>>(static_cast<const uint4*>(bitmap), nq,
                                                       static_cast<int32_t*>(blocks));
   });
 }

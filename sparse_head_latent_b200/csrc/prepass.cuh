@@ -20,7 +20,8 @@
 //                             shared-memory atomics build the row's bits,
 //                             then the row's words are written for every
 //                             causal block (rows past T get zeros)
-//   topk_block_list_kernel    one CTA per (tile group, batch): OR of each
+//   topk_block_list_kernel    one CTA per (tile group, batch), a warp per key
+//                             block: OR of each
 //                             block's bits over the group's tiles,
 //                             ballot-compacted into the group's list
 // No global atomics; the result is deterministic.
@@ -55,7 +56,20 @@ topk_bitmap_rows_kernel(const int32_t* __restrict__ topk_idx, int B, int T, int 
   __syncwarp();
   if (s < T) {
     const int32_t* idx = topk_idx + (static_cast<int64_t>(b) * T + s) * k;
-    for (int i = lane; i < k; i += 32) {
+    int i0 = 0;
+    if ((k & 3) == 0 && (reinterpret_cast<uintptr_t>(topk_idx) & 15u) == 0) {
+      // 16-byte loads, two per lane per round, issued before the atomics so
+      // that several are in flight (the row is 4k bytes).
+      for (; i0 + 256 <= k; i0 += 256) {
+        const int4 u = __ldg(reinterpret_cast<const int4*>(idx + i0) + lane);
+        const int4 v = __ldg(reinterpret_cast<const int4*>(idx + i0 + 128) + lane);
+        const int32_t t[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (t[j] >= 0 && t[j] <= s) atomicOr(&bits[t[j] >> 5], 1u << (t[j] & 31));
+      }
+    }
+    for (int i = i0 + lane; i < k; i += 32) {
       const int32_t t = __ldg(idx + i);
       if (t >= 0 && t <= s) atomicOr(&bits[t >> 5], 1u << (t & 31));
     }
@@ -65,7 +79,9 @@ topk_bitmap_rows_kernel(const int32_t* __restrict__ topk_idx, int B, int T, int 
   for (int w = lane; w < nwords; w += 32) bm[(static_cast<int64_t>(w >> 2) * 128 + r) * 4 + (w & 3)] = bits[w];
 }
 
-__global__ void __launch_bounds__(128)
+constexpr int kBlockListWarps = 16;
+
+__global__ void __launch_bounds__(32 * kBlockListWarps)
 topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __restrict__ blocks) {
   __shared__ uint32_t flags[MLA_MAX_T / 128];
   const int g = blockIdx.x, b = blockIdx.y;
@@ -73,7 +89,7 @@ topk_block_list_kernel(const uint4* __restrict__ bitmap, int nq, int32_t* __rest
   const int last = min(q0 + 3, nq - 1);     // highest key block a tile of the group can see
   const int last_a = min(q0 + 1, nq - 1);   // highest one of the group's first two tiles
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int kb = warp; kb <= last; kb += 4) {
+  for (int kb = warp; kb <= last; kb += kBlockListWarps) {
     uint32_t acc = 0;
     for (int qt = q0; qt <= last; ++qt) {
       if (kb > qt) continue;  // outside this tile's causal triangle
