@@ -48,7 +48,9 @@ KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "gemm_m64.cuh", "quant.cu
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default 200; 2000 for the decode step, so that its timed region lasts "
+                        "long enough for the clock samples)")
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--config", type=int, default=1)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -66,7 +68,10 @@ def parse_args(argv=None):
                         "split over the ranks and the partial outputs all-reduced (strong scaling)")
     p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
                    help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
-    return p.parse_args(argv)
+    args = p.parse_args(argv)
+    if args.steps is None:
+        args.steps = 2000 if args.mode == "decode" and args.impl == "ours" else 200
+    return args
 
 
 def workload(args):
@@ -155,7 +160,7 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 100):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.gpu, self.period = gpu_index, period_ms
         self.proc = None
         self.lines = []
@@ -580,9 +585,10 @@ def run_decode(args, local):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
-    # Per-kernel times from an eager, profiled run.
+    # Per-kernel times from an eager, profiled run of a few of the steps.
+    prof_steps = min(args.steps, 50)
     mla.mla_profile_begin()
-    for _ in range(args.steps):
+    for _ in range(prof_steps):
         step()
     torch.cuda.synchronize(dev)
     prof = mla.mla_profile_end()
@@ -651,9 +657,9 @@ def run_decode(args, local):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                      "traffic": None, "peak_source": f"{src} HBM copy bandwidth",
                      "bytes_per_step": compulsory},
-        "per_kernel": per, "per_kernel_source": "eager profiled run of the same steps",
+        "per_kernel": per, "per_kernel_source": f"eager profiled run of {prof_steps} of the steps",
         "timing": "CUDA graph replay of the whole decode step",
-        "gpu_launches": sum(c for _, c in prof.values()),
+        "gpu_launches": int(round(sum(c for _, c in prof.values()) / prof_steps * args.steps)),
         "e2e": {"value": round(B / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "clocks": clocks.summary(t_wall0, t_wall1),

@@ -17,6 +17,11 @@
 // For 64 < M <= 128 the tiles have 128 rows (UMMA M = 128), so that the
 // weight is still streamed once.
 //
+// The same kernel runs the decode step's per-head GEMMs (the absorption of
+// q_nope into W_UK and the un-absorption of o_lat through W_UV) as a batch:
+// item z of the batch reads A columns, B rows and writes C columns at offsets
+// z * step (M64Batch), stores bf16 directly, and may read B K-major.
+//
 // Roles (192 threads, one CTA per SM, persistent over the work items):
 //   warp 0      TMA producer
 //   warp 1      tensor-memory allocator (256 columns: two accumulators) and
@@ -30,10 +35,15 @@
 
 namespace mla {
 
-template <int BM_>
+// B_MN_MAJOR_: B stored [K, N] (N contiguous; two 64-column boxes per
+// stage) or [N, K] (K contiguous; one 128-row box). OUT_BF16_: items write
+// bf16 C columns directly instead of fp32 partial planes.
+template <int BM_, bool B_MN_MAJOR_ = true, bool OUT_BF16_ = false>
 struct GemmM64Cfg {
   static_assert(BM_ == 64 || BM_ == 128, "row tile");
   static constexpr int BM = BM_, BN = 128, BK = 64;
+  static constexpr bool B_MN_MAJOR = B_MN_MAJOR_;
+  static constexpr bool OUT_BF16 = OUT_BF16_;
   static constexpr int STAGES = BM_ == 64 ? 8 : 6;
   static constexpr int A_BYTES = BM * BK * 2;   // 8 or 16 KB
   static constexpr int B_BYTES = BK * BN * 2;   // 16 KB: two [64 K rows x 64 columns] boxes
@@ -45,11 +55,22 @@ struct GemmM64Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// Work item i = ((s * num_n) + nt) * num_m + mt.
+// Item z of the z dimension (a K range of a split-K GEMM, or a head of a
+// batch): A columns from z * a_step, B rows from b_row0 + z * b_step (K rows
+// for an N-major B, N rows for a K-major one), output fp32 plane z of `part`
+// [count][M][N], or bf16 columns from z * c_step of `out` (row pitch ldc).
+struct M64Batch {
+  int count;
+  int a_step, b_row0, b_step;
+  int c_step, ldc;
+};
+
+// Work item i = ((z * num_n) + nt) * num_m + mt; each item runs K columns of A.
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                       int N, int K, int splits, float* __restrict__ part, int* err) {
+                       int N, int K, const M64Batch bt, float* __restrict__ part, __nv_bfloat16* __restrict__ out,
+                       int* err) {
   constexpr int BK = Cfg::BK, S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,9 +110,8 @@ gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
   const int num_m = (M + Cfg::BM - 1) / Cfg::BM;
   const int num_n = N / Cfg::BN;
-  const int items = num_m * num_n * splits;
-  const int ks = K / splits;  // a multiple of BK (host-checked)
-  const int num_kb = ks / BK;
+  const int items = num_m * num_n * bt.count;
+  const int num_kb = K / BK;  // K a multiple of BK (host-checked)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -110,10 +130,15 @@ gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
           const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t sb = sa + Cfg::A_BYTES;
-          const int k = sp * ks + kb * BK;
-          tma_load_2d(sa, &tmA, fb, k, mt * Cfg::BM);  // rows past M read as zero
-          tma_load_2d(sb, &tmB, fb, nt * Cfg::BN, k);
-          tma_load_2d(sb + BK * 128, &tmB, fb, nt * Cfg::BN + 64, k);
+          const int k = kb * BK;
+          tma_load_2d(sa, &tmA, fb, sp * bt.a_step + k, mt * Cfg::BM);  // rows past M read as zero
+          if constexpr (Cfg::B_MN_MAJOR) {
+            const int kr = bt.b_row0 + sp * bt.b_step + k;
+            tma_load_2d(sb, &tmB, fb, nt * Cfg::BN, kr);
+            tma_load_2d(sb + BK * 128, &tmB, fb, nt * Cfg::BN + 64, kr);
+          } else {
+            tma_load_2d(sb, &tmB, fb, k, bt.b_row0 + sp * bt.b_step + nt * Cfg::BN);  // box 64 K x 128 N rows
+          }
         }
       }
       if (!ok) spin_ns(2000000);  // let issued loads land before the CTA can exit
@@ -121,7 +146,7 @@ gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- UMMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, 0, 1);
+      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, 0, Cfg::B_MN_MAJOR ? 1 : 0);
       int it = 0, t = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++t) {
@@ -143,7 +168,9 @@ gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           const uint32_t sb = sa + Cfg::A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_ss(d, smem_desc_sw128(sa + k * 32, 16, 1024), smem_desc_sw128(sb + k * 16 * 128, BK * 128, 1024),
+            umma_ss(d, smem_desc_sw128(sa + k * 32, 16, 1024),
+                    Cfg::B_MN_MAJOR ? smem_desc_sw128(sb + k * 16 * 128, BK * 128, 1024)
+                                    : smem_desc_sw128(sb + k * 32, 16, 1024),
                     idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(empty0 + 8 * s);
         }
@@ -168,17 +195,27 @@ gemm_m64_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * Cfg::BN;
       const int row = mt * Cfg::BM + RPW * q + static_cast<int>(lane);
-      float* dst = part + (static_cast<size_t>(sp) * M + row) * N + nt * Cfg::BN;
 #pragma unroll 1
       for (int c = 0; c < Cfg::BN; c += 32) {
         uint32_t v[32];
         tmem_ld32(tb + c, v);
         if (static_cast<int>(lane) < RPW && row < M) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c);
+          if constexpr (Cfg::OUT_BF16) {
+            uint4* d4 = reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * bt.ldc + sp * bt.c_step +
+                                                 nt * Cfg::BN + c);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+          } else {
+            float4* d4 = reinterpret_cast<float4*>(part + (static_cast<size_t>(sp) * M + row) * N + nt * Cfg::BN + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
         }
       }
       tc_fence_before();

@@ -36,6 +36,10 @@ using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B store
 using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
 using GemmM64 = mla::GemmM64Cfg<64>;     // decode's output projection, M <= 64
 using GemmM128 = mla::GemmM64Cfg<128>;   // and 64 < M <= 256 (128-row tiles)
+using GemmM64Abs = mla::GemmM64Cfg<64, true, true>;     // decode's q_nope x W_UK per head, bf16 out
+using GemmM128Abs = mla::GemmM64Cfg<128, true, true>;
+using GemmM64Unabs = mla::GemmM64Cfg<64, false, true>;  // decode's o_lat x W_UV^T per head, bf16 out
+using GemmM128Unabs = mla::GemmM64Cfg<128, false, true>;
 using Gemm8Kvb = mla::Gemm8Cfg<false>;              // e4m3 latent x e4m3 W_kvb^T
 using Gemm8KvbAttn = mla::Gemm8Cfg<false, true>;    // same, v tiles written as f16 for the attention
 using Gemm8Wo = mla::Gemm8Cfg<true>;           // e4m3 attn x e4m3 W_o (B stored [K, N])
@@ -132,6 +136,14 @@ int device_state(DeviceState** out) {
                                       GemmM64::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM128::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64Abs>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM64Abs::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128Abs>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM128Abs::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64Unabs>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM64Unabs::SMEM_BYTES) == cudaSuccess;
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128Unabs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      GemmM128Unabs::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AbsSmem::BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::sparse_mla_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -506,6 +518,25 @@ int launch_gemm8_wo(const DeviceState* ds, int M, int H, const void* attn8, cons
   return launch_gemm8_pair<Gemm8Wo>(ds->pairs8_wo, ta, tb, tc, M, N, K, sc, ds->err, 4, st);
 }
 
+// One launch of the few-row GEMM: 64-row tiles for M <= 64, else 128-row
+// tiles (Cfg64 / Cfg128); K columns of A per work item.
+template <class Cfg64, class Cfg128>
+int launch_m64(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+               const mla::M64Batch& bt, float* part, void* out, int cls, cudaStream_t st) {
+  const int bm = M <= 64 ? 64 : 128;
+  const int items = ((M + bm - 1) / bm) * (N / Cfg64::BN) * bt.count;
+  const int grid = items < ds->sms ? items : ds->sms;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  return timed_launch(cls, st, [&] {
+    if (bm == 64)
+      mla::gemm_m64_splitk_kernel<Cfg64><<<grid, Cfg64::THREADS, Cfg64::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt, part,
+                                                                                         o, ds->err);
+    else
+      mla::gemm_m64_splitk_kernel<Cfg128><<<grid, Cfg128::THREADS, Cfg128::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt,
+                                                                                            part, o, ds->err);
+  });
+}
+
 // Output projection of M <= 256 rows as a split-K GEMM (M = 64 UMMA tiles):
 // fp32 partial outputs per K range into `part`, then summed into `out`.
 int launch_gemm_wo_m64(const DeviceState* ds, int M, int H, const void* attn, const void* wo, float* part,
@@ -517,16 +548,9 @@ int launch_gemm_wo_m64(const DeviceState* ds, int M, int H, const void* attn, co
   if (!map_2d(&ta, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, bm) ||
       !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64))
     return MLA_ERR_CUDA;
-  const int items = ((M + bm - 1) / bm) * (N / GemmM64::BN) * splits;
-  const int grid = items < ds->sms ? items : ds->sms;
-  int rc = timed_launch(4, st, [&] {
-    if (bm == 64)
-      mla::gemm_m64_splitk_kernel<GemmM64><<<grid, GemmM64::THREADS, GemmM64::SMEM_BYTES, st>>>(
-          ta, tb, M, N, K, splits, part, ds->err);
-    else
-      mla::gemm_m64_splitk_kernel<GemmM128><<<grid, GemmM128::THREADS, GemmM128::SMEM_BYTES, st>>>(
-          ta, tb, M, N, K, splits, part, ds->err);
-  });
+  const int ks = K / splits;
+  const mla::M64Batch bt = {splits, ks, 0, ks, 0, 0};
+  int rc = launch_m64<GemmM64, GemmM128>(ds, ta, tb, M, N, ks, bt, part, nullptr, 4, st);
   if (rc != MLA_OK) return rc;
   const int64_t quads = static_cast<int64_t>(M) * N / 4;
   return timed_launch(4, st, [&] {
@@ -628,12 +652,23 @@ int launch_decode_lists(const mla_dims& d, const int32_t* topk, int kpad, int32_
   });
 }
 
+// Up to this many rows the per-head GEMMs run on the few-row kernel (64- or
+// 128-row UMMA tiles, one CTA per item), beyond it on the CTA-pair GEMM.
+constexpr int kFewRows = 256;
+
 // q_abs[r, h, :] = q[r, h, 0:128] . W_kvb[h*256 + (0..127), :] for `rows`
 // consecutive rows: one GEMM per head (M = rows, N = 512, K = 128).
 int launch_gemm_absorb(const DeviceState* ds, int H, int rows, const void* q_rows, const void* wk, void* qabs,
                        cudaStream_t st) {
   CUtensorMap ta, tb, tc;
   const uint64_t qw = static_cast<uint64_t>(H) * (kDn + kDr);
+  if (rows <= kFewRows) {
+    if (!map_2d(&ta, q_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qw, rows, qw * 2, 64, rows <= 64 ? 64 : 128) ||
+        !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64, 64))
+      return MLA_ERR_CUDA;
+    const mla::M64Batch bt = {H, kDn + kDr, 0, kDn + kDv, kL, H * kL};
+    return launch_m64<GemmM64Abs, GemmM128Abs>(ds, ta, tb, rows, kL, kDn, bt, nullptr, qabs, 6, st);
+  }
   if (!map_2d(&ta, q_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qw, rows, qw * 2, 64, 128) ||
       !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64, 64) ||
       !map_2d(&tc, qabs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
@@ -648,6 +683,15 @@ int launch_gemm_absorb(const DeviceState* ds, int H, int rows, const void* q_row
 int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* olat, const void* wk, void* attn_rows,
                          cudaStream_t st) {
   CUtensorMap ta, tb, tc;
+  if (rows <= kFewRows) {
+    if (!map_2d(&ta, olat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
+                static_cast<uint64_t>(H) * kL * 2, 64, rows <= 64 ? 64 : 128) ||
+        !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64,
+                128))
+      return MLA_ERR_CUDA;
+    const mla::M64Batch bt = {H, kL, kDn, kDn + kDv, kDv, H * kDv};
+    return launch_m64<GemmM64Unabs, GemmM128Unabs>(ds, ta, tb, rows, kDv, kL, bt, nullptr, attn_rows, 6, st);
+  }
   if (!map_2d(&ta, olat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
               static_cast<uint64_t>(H) * kL * 2, 64, 128) ||
       !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64,

@@ -28,6 +28,9 @@ DECODE_CASES = {
     # several CTAs and the partial results combined
     "split_keys": dict(B=2, T=3000, H=4, topk=1024),
     "split_keys_64_heads": dict(B=1, T=2100, H=64, topk=1024),
+    # more than 64 sequences: the per-head and output GEMMs take 128-row
+    # tiles, the second one partly past the last row
+    "batch_100": dict(B=100, T=40, H=4, topk=12),
 }
 
 
