@@ -34,7 +34,7 @@ using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as 
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
 using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
-using GemmM64 = mla::GemmM64Cfg<64>;     // decode's output projection, M <= 64
+using GemmM64 = mla::GemmM64Cfg<64>;     // decode's output projection (stream-K), M <= 64
 using GemmM128 = mla::GemmM64Cfg<128>;   // and 64 < M <= 256 (128-row tiles)
 using GemmM64Abs = mla::GemmM64Cfg<64, true, true>;     // decode's q_nope x W_UK per head, bf16 out
 using GemmM128Abs = mla::GemmM64Cfg<128, true, true>;
@@ -132,17 +132,17 @@ int device_state(DeviceState** out) {
         st.pairs8_wo = max_pairs(mla::gemm_e4m3_tc2_kernel<Gemm8Wo>, Gemm8Wo::SMEM_BYTES, Gemm8Wo::THREADS);
         ok = st.pairs8_kvb > 0 && st.pairs8_wo > 0;
       }
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       GemmM64::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128>,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM128>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM128::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64Abs>,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM64Abs>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM64Abs::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128Abs>,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM128Abs>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM128Abs::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM64Unabs>,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM64Unabs>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GemmM64Unabs::SMEM_BYTES) == cudaSuccess;
-      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_splitk_kernel<GemmM128Unabs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      ok = ok && cudaFuncSetAttribute(mla::gemm_m64_kernel<GemmM128Unabs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       GemmM128Unabs::SMEM_BYTES) == cudaSuccess;
       ok = ok && cudaFuncSetAttribute(mla::absorbed_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       mla::AbsSmem::BYTES) == cudaSuccess;
@@ -249,8 +249,7 @@ struct WsLayout {
   size_t lat8 = kNone, lat8_s = kNone;    // e4m3 activations: quantized latent and its scales
   size_t attn8 = kNone, attn8_s = kNone;  // e4m3 activations: quantized attention rows and scales
   int parts = 1;                          // decode: CTAs per (sequence, 64-head group)
-  int wo_splits = 1;                      // decode: K ranges of the output projection
-  size_t wo_part = kNone;                 // decode: their fp32 partial outputs [wo_splits, B, 7168]
+  size_t wo_part = kNone;                 // decode: stream-K partial tiles of the output projection
   int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
   int abs_chunk = 0;   // absorbed rows processed per pass
   int kpad = 0;        // pitch of the per-row key lists
@@ -264,6 +263,7 @@ constexpr int kAbsChunkRows = 2048;
 // SM count the decode split is planned for (the workspace size cannot depend
 // on the device; a different count only changes how full the waves are).
 constexpr int kSmsForSplit = 148;
+constexpr int kStreamKCtas = 256;  // upper bound on the stream-K grid (the SM count)
 // Cost model for MLA_PATH_AUTO: a tile group goes absorbed when its middle
 // row's causal prefix exceeds this many times the selection size. Measured
 // on B200 at T = 32768, H = 128, top-k 2048: the block-dense kernel costs
@@ -356,11 +356,12 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
       w.part_ml = take(B * w.parts * H * 8);
       w.part_o = take(B * w.parts * H * kL * 2);
     }
-    // The output projection of up to 256 rows runs as a split-K GEMM with
-    // M = 64 tiles: K = 128 H is cut into ranges of whole 64-deep blocks.
+    // The output projection of up to 256 rows runs as a stream-K GEMM with
+    // 64- or 128-row tiles: one fp32 partial tile per (CTA, tile) segment.
     if (d.B <= 256) {
-      w.wo_splits = (2 * d.H) % 8 == 0 ? 8 : (2 * d.H) % 4 == 0 ? 4 : 2;
-      w.wo_part = take(static_cast<size_t>(w.wo_splits) * B * kD * 4);
+      const int bm = d.B <= 64 ? 64 : 128;
+      const size_t tiles = static_cast<size_t>((d.B + bm - 1) / bm) * (kD / 128);
+      w.wo_part = take((kStreamKCtas + tiles) * bm * 128 * 4);
     }
   }
   const bool dec = entry == MLA_ENTRY_DECODE;
@@ -519,43 +520,45 @@ int launch_gemm8_wo(const DeviceState* ds, int M, int H, const void* attn8, cons
 }
 
 // One launch of the few-row GEMM: 64-row tiles for M <= 64, else 128-row
-// tiles (Cfg64 / Cfg128); K columns of A per work item.
+// tiles (Cfg64 / Cfg128); K columns of A per batch item, or the stream-K
+// split of one GEMM over `grid` CTAs.
 template <class Cfg64, class Cfg128>
 int launch_m64(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
-               const mla::M64Batch& bt, float* part, void* out, int cls, cudaStream_t st) {
+               const mla::M64Batch& bt, int grid, float* part, void* out, int cls, cudaStream_t st) {
   const int bm = M <= 64 ? 64 : 128;
-  const int items = ((M + bm - 1) / bm) * (N / Cfg64::BN) * bt.count;
-  const int grid = items < ds->sms ? items : ds->sms;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   return timed_launch(cls, st, [&] {
     if (bm == 64)
-      mla::gemm_m64_splitk_kernel<Cfg64><<<grid, Cfg64::THREADS, Cfg64::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt, part,
+      mla::gemm_m64_kernel<Cfg64><<<grid, Cfg64::THREADS, Cfg64::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt, part,
                                                                                          o, ds->err);
     else
-      mla::gemm_m64_splitk_kernel<Cfg128><<<grid, Cfg128::THREADS, Cfg128::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt,
+      mla::gemm_m64_kernel<Cfg128><<<grid, Cfg128::THREADS, Cfg128::SMEM_BYTES, st>>>(ta, tb, M, N, K, bt,
                                                                                             part, o, ds->err);
   });
 }
 
-// Output projection of M <= 256 rows as a split-K GEMM (M = 64 UMMA tiles):
-// fp32 partial outputs per K range into `part`, then summed into `out`.
+// Output projection of M <= 256 rows as a stream-K GEMM (M = 64 or 128 UMMA
+// tiles): every CTA takes an equal share of the tiles' k-blocks and writes
+// one fp32 partial tile per tile it touches into `part` (room for
+// kStreamKCtas + tiles of them); a second kernel sums them into `out`.
 int launch_gemm_wo_m64(const DeviceState* ds, int M, int H, const void* attn, const void* wo, float* part,
-                       int splits, void* out, cudaStream_t st) {
+                       void* out, cudaStream_t st) {
   const int N = kD, K = H * kDv;
-  if ((K / splits) % GemmM64::BK != 0) return MLA_ERR_SHAPE;
   const int bm = M <= 64 ? 64 : 128;
   CUtensorMap ta, tb;
   if (!map_2d(&ta, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, bm) ||
       !map_2d(&tb, wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, K, static_cast<uint64_t>(N) * 2, 64, 64))
     return MLA_ERR_CUDA;
-  const int ks = K / splits;
-  const mla::M64Batch bt = {splits, ks, 0, ks, 0, 0};
-  int rc = launch_m64<GemmM64, GemmM128>(ds, ta, tb, M, N, ks, bt, part, nullptr, 4, st);
+  const int64_t units = static_cast<int64_t>((M + bm - 1) / bm) * (N / GemmM64::BN) * (K / GemmM64::BK);
+  int grid = ds->sms < kStreamKCtas ? ds->sms : kStreamKCtas;
+  if (units < grid) grid = static_cast<int>(units);
+  const mla::M64Batch bt = {1, 0, 0, 0, 0, 0};
+  int rc = launch_m64<GemmM64, GemmM128>(ds, ta, tb, M, N, K, bt, grid, part, nullptr, 4, st);
   if (rc != MLA_OK) return rc;
-  const int64_t quads = static_cast<int64_t>(M) * N / 4;
+  const int blocks = ((M + bm - 1) / bm) * (N / GemmM64::BN) * (bm / mla::kSumRows);
   return timed_launch(4, st, [&] {
-    mla::sum_splits_kernel<<<static_cast<unsigned>((quads + 255) / 256), 256, 0, st>>>(
-        part, M, N, splits, static_cast<__nv_bfloat16*>(out));
+    mla::sum_segments_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, M, N, K, bm, grid,
+                                                                            static_cast<__nv_bfloat16*>(out), ds->err);
   });
 }
 
@@ -667,7 +670,9 @@ int launch_gemm_absorb(const DeviceState* ds, int H, int rows, const void* q_row
         !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64, 64))
       return MLA_ERR_CUDA;
     const mla::M64Batch bt = {H, kDn + kDr, 0, kDn + kDv, kL, H * kL};
-    return launch_m64<GemmM64Abs, GemmM128Abs>(ds, ta, tb, rows, kL, kDn, bt, nullptr, qabs, 6, st);
+    const int items = (rows <= 64 ? 1 : (rows + 127) / 128) * (kL / 128) * H;
+    return launch_m64<GemmM64Abs, GemmM128Abs>(ds, ta, tb, rows, kL, kDn, bt, items < ds->sms ? items : ds->sms,
+                                               nullptr, qabs, 6, st);
   }
   if (!map_2d(&ta, q_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qw, rows, qw * 2, 64, 128) ||
       !map_2d(&tb, wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kL, static_cast<uint64_t>(H) * (kDn + kDv), kL * 2, 64, 64) ||
@@ -690,7 +695,9 @@ int launch_gemm_unabsorb(const DeviceState* ds, int H, int rows, const void* ola
                 128))
       return MLA_ERR_CUDA;
     const mla::M64Batch bt = {H, kL, kDn, kDn + kDv, kDv, H * kDv};
-    return launch_m64<GemmM64Unabs, GemmM128Unabs>(ds, ta, tb, rows, kDv, kL, bt, nullptr, attn_rows, 6, st);
+    const int items = (rows <= 64 ? 1 : (rows + 127) / 128) * H;
+    return launch_m64<GemmM64Unabs, GemmM128Unabs>(ds, ta, tb, rows, kDv, kL, bt, items < ds->sms ? items : ds->sms,
+                                                   nullptr, attn_rows, 6, st);
   }
   if (!map_2d(&ta, olat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(H) * kL, rows,
               static_cast<uint64_t>(H) * kL * 2, 64, 128) ||
@@ -886,9 +893,8 @@ int run_decode(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
     if ((rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st)) != MLA_OK) return rc;
     wo = dq;
   }
-  if (lay.wo_splits > 1)
-    return launch_gemm_wo_m64(ds, d.B, d.H, attn, wo, reinterpret_cast<float*>(ws_at(ws, lay.wo_part)),
-                              lay.wo_splits, out, st);
+  if (lay.wo_part != kNone)
+    return launch_gemm_wo_m64(ds, d.B, d.H, attn, wo, reinterpret_cast<float*>(ws_at(ws, lay.wo_part)), out, st);
   return launch_gemm_wo(ds, d.B, d.H, attn, wo, out, st);
 }
 
