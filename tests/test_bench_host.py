@@ -91,3 +91,12 @@ def test_cpu_baseline_sample_is_bounded():
     d = bench.cpu_baseline(x, 0.5)
     assert d["kind"] == "oracle" and d["cores"] == 1 and d["value"] > 0
     assert d["seconds"] < 5
+
+
+def test_step_defaults_per_mode():
+    # The decode step is ~0.2 ms, so its default timed region (2000 graph
+    # replays) still spans many clock samples; the other modes keep 200.
+    assert bench.parse_args([]).steps == 200
+    assert bench.parse_args(["--mode", "decode"]).steps == 2000
+    assert bench.parse_args(["--mode", "decode", "--impl", "reference"]).steps == 200
+    assert bench.parse_args(["--mode", "decode", "--steps", "7"]).steps == 7
