@@ -66,6 +66,9 @@ def parse_args(argv=None):
     p.add_argument("--parallel", choices=["sequences", "heads"], default="sequences",
                    help="N > 1: independent sequences per rank (weak scaling) or one problem with its heads "
                         "split over the ranks and the partial outputs all-reduced (strong scaling)")
+    p.add_argument("--selections", type=int, default=1,
+                   help="decode: rotate through this many different top-k selections, one per step (a device "
+                        "copy of the next selection precedes every timed step); 1 repeats the same selection")
     p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
                    help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
     args = p.parse_args(argv)
@@ -573,6 +576,11 @@ def run_decode(args, local):
     x = synth.make_decode_inputs(B, T, H, k, seed=11)
     dev = torch.device("cuda", local)
     g = {n: v.to(dev) for n, v in x.tensors().items()}
+    # Selections to rotate through (set 0 is the inputs' own): with a single
+    # repeated selection the gathered latent rows of one step can still be in
+    # L2 at the next.
+    nsel = max(1, args.selections)
+    sel_sets = torch.stack([x.topk_idx] + [synth.decode_topk(B, T, k, 11 + r) for r in range(1, nsel)]).to(dev)
     dims = mla.make_dims(B, T, H, k, False)
     ws = torch.empty(mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_DECODE, True), dtype=torch.uint8, device=dev)
     out = torch.empty(B, 7168, dtype=torch.bfloat16, device=dev)
@@ -605,7 +613,9 @@ def run_decode(args, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        if nsel > 1:
+            g["topk_idx"].copy_(sel_sets[i % nsel], non_blocking=True)
         graph.replay()
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -614,6 +624,7 @@ def run_decode(args, local):
     if mla.mla_device_status(stream) != 0:
         raise RuntimeError("device error in the timed region")
     ms = e0.elapsed_time(e1) / args.steps
+    g["topk_idx"].copy_(sel_sets[0])
     # End to end: every step copies its new inputs from pinned host memory --
     # the queries, the selections and the new position's latent and rope rows
     # (the cache itself stays resident) -- replays the step and copies the
@@ -651,7 +662,10 @@ def run_decode(args, local):
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; no checkpoint)",
         "config": {"workload": f"decode_B{B}_T{T}", "B": B, "T": T, "H": H, "topk": k, "weights": "bf16",
-                   "l2": "no flush: W_o alone (235 MB) exceeds the 126 MB L2"},
+                   "selections": nsel,
+                   "l2": "no flush: W_o alone (235 MB) exceeds the 126 MB L2; "
+                         + ("the same selection every step (its gathered rows can stay in L2)" if nsel == 1 else
+                            f"{nsel} selections in rotation, a device copy of the next one inside each timed step")},
         "algorithmic_gflop_per_step": round(flops / 1e9, 3),
         "roofline": {"kernel": "whole decode step", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),

@@ -14,6 +14,7 @@ from .inputs import (  # noqa: F401
     SOFTMAX_SCALE,
     DecodeInputs,
     MlaInputs,
+    decode_topk,
     make_decode_inputs,
     make_inputs,
     make_topk,

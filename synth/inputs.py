@@ -237,21 +237,26 @@ def make_decode_inputs(B: int, T: int, H: int, topk: Optional[int], seed: int, f
         wk = _randn_bf16((H * (D_NOPE + D_V), D_LATENT), g(_TID_WKVB), std_kvb)
         wo = _randn_bf16((H * D_V, D_MODEL), g(_TID_WO), std_o)
         sk = so = None
-    tk = None
-    if topk is not None:
-        gt = g(_TID_TOPK)
-        n = min(int(topk), T)
-        rows = []
-        for _ in range(B):
-            others = torch.randperm(T - 1, generator=gt)[: n - 1] if n > 1 else torch.empty(0, dtype=torch.int64)
-            sel = torch.cat([torch.tensor([T - 1]), others])
-            sel = sel[torch.randperm(n, generator=gt)]
-            if int(topk) > n:  # more entries than positions: out-of-range fillers select nothing
-                sel = torch.cat([sel, torch.arange(T, T + int(topk) - n)])
-            rows.append(sel)
-        tk = torch.stack(rows).to(torch.int32).contiguous()
+    tk = decode_topk(B, T, topk, seed) if topk is not None else None
     return DecodeInputs(B=B, T=T, H=H, topk=topk, fp8=fp8, scale=SOFTMAX_SCALE, q=q, kv_latent=lat, k_pe=kpe,
                         W_kvb=wk, W_kvb_scale=sk, W_o=wo, W_o_scale=so, topk_idx=tk)
+
+
+def decode_topk(B: int, T: int, topk: int, seed: int) -> torch.Tensor:
+    """The selection of make_decode_inputs (same seed, same bytes): per
+    sequence, s = T - 1 plus min(k, T) - 1 distinct positions of [0, s) in a
+    shuffled order, padded with out-of-range fillers when k > T. int32 [B, k]."""
+    gt = _gen(seed, _TID_TOPK)
+    n = min(int(topk), T)
+    rows = []
+    for _ in range(B):
+        others = torch.randperm(T - 1, generator=gt)[: n - 1] if n > 1 else torch.empty(0, dtype=torch.int64)
+        sel = torch.cat([torch.tensor([T - 1]), others])
+        sel = sel[torch.randperm(n, generator=gt)]
+        if int(topk) > n:  # more entries than positions: out-of-range fillers select nothing
+            sel = torch.cat([sel, torch.arange(T, T + int(topk) - n)])
+        rows.append(sel)
+    return torch.stack(rows).to(torch.int32).contiguous()
 
 
 def sample_rows(B: int, T: int, k: Optional[int], n_random: int, seed: int,

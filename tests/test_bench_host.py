@@ -100,3 +100,15 @@ def test_step_defaults_per_mode():
     assert bench.parse_args(["--mode", "decode"]).steps == 2000
     assert bench.parse_args(["--mode", "decode", "--impl", "reference"]).steps == 200
     assert bench.parse_args(["--mode", "decode", "--steps", "7"]).steps == 7
+
+
+def test_decode_selection_sets():
+    # Set 0 of the decode bench's rotation is the inputs' own selection; the
+    # others follow the same rule (s = T-1 plus distinct earlier positions).
+    d = synth.make_decode_inputs(3, 50, 2, 16, seed=11)
+    assert torch.equal(synth.decode_topk(3, 50, 16, 11), d.topk_idx)
+    other = synth.decode_topk(3, 50, 16, 12)
+    assert not torch.equal(other, d.topk_idx)
+    for row in other:
+        vals = sorted(row.tolist())
+        assert len(set(vals)) == 16 and vals[-1] == 49 and vals[0] >= 0
