@@ -182,3 +182,24 @@ def test_dims_struct_matches_header():
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     names = re.findall(r"\b([A-Za-z_]+)\s*[,;]", body)
     assert names == [f for f, _ in MlaDims._fields_]
+
+
+def test_workspace_sizes_decode(lib):
+    # q_abs and o_lat (B x H x 512 bf16 each), the key lists (k rounded up to
+    # 64, int32) and counts, the un-absorbed rows (B x H x 128 bf16) and, up
+    # to 256 sequences, the output projection's stream-K partial tiles: one
+    # fp32 tile of 64 (128 above 64 sequences) x 128 per slot, for at most
+    # 256 CTAs plus one slot per tile (7168 / 128 = 56 column tiles per row tile).
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    H, k = 4, 300
+    kpad = 320  # five 64-key blocks: too few to split a sequence's keys over CTAs
+    for B, bm, m_tiles in ((64, 64, 1), (100, 128, 1), (200, 128, 2)):
+        d = MlaDims(B, 1000, H, 128, 64, 128, 512, 7168, k, 0, 0, 0)
+        want = (2 * up(B * H * 512 * 2) + up(B * kpad * 4) + up(B * 4) + up(B * H * 128 * 2)
+                + up((256 + m_tiles * 56) * bm * 128 * 4))
+        assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_DECODE, True) == want, B
+    # beyond 256 sequences the output projection runs on the pair GEMM: no partial tiles
+    B = 300
+    d = MlaDims(B, 1000, H, 128, 64, 128, 512, 7168, k, 0, 0, 0)
+    assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_DECODE, True) == (
+        2 * up(B * H * 512 * 2) + up(B * kpad * 4) + up(B * 4) + up(B * H * 128 * 2))
