@@ -244,6 +244,46 @@ def oracle_unit(x, rng):
     return dt, flops
 
 
+DECODE_METRIC = "sparse MLA decode tokens/s (one new position per sequence, absorbed form)"
+
+
+def decode_unit_problem(q_row, lat_b, kpe_b, W_kvb, W_o, sel, h, scale):
+    """The oracle's problem for one (sequence, head) of a decode step: the
+    head's query row attending its selected cache positions `sel` (ascending),
+    laid out as a causal prefill of n = len(sel) positions whose last row is
+    the query, so that it attends exactly those keys in the same ascending
+    order; the head's W_kvb rows and W_o rows. Its output row is the head's
+    share of the decode output (the shares sum over heads)."""
+    from types import SimpleNamespace
+    n = int(sel.numel())
+    q = torch.zeros(1, n, 1, q_row.shape[-1], dtype=q_row.dtype)
+    q[0, n - 1, 0] = q_row
+    return SimpleNamespace(B=1, T=n, H=1, fp8=False, scale=scale, topk_idx=None, q=q,
+                           kv_latent=lat_b[sel].unsqueeze(0).contiguous(),
+                           k_pe=kpe_b[sel].unsqueeze(0).contiguous(),
+                           W_kvb=W_kvb[h * 256:(h + 1) * 256], W_kvb_scale=None,
+                           W_o=W_o[h * 128:(h + 1) * 128], W_o_scale=None)
+
+
+def oracle_decode_unit(x, rng):
+    """One sampled unit of the decode workload for the CPU oracle: a random
+    (sequence, head): the fp64 up-projection of its selected cache rows for
+    that head, the masked softmax, the value mix and the head's slice of
+    W_o. Returns seconds."""
+    import oracle
+    b = int(rng.integers(0, x.B))
+    h = int(rng.integers(0, x.H))
+    if x.topk_idx is None:
+        sel = torch.arange(x.T)
+    else:
+        tk = x.topk_idx[b]
+        sel = torch.unique(tk[(tk >= 0) & (tk < x.T)])
+    y = decode_unit_problem(x.q[b, h], x.kv_latent[b], x.k_pe[b], x.W_kvb, x.W_o, sel, h, x.scale)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(y, [y.T - 1])
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(x, budget_s: float, seed: int = 7):
     rng = np.random.default_rng(seed)
     tot_t, tot_f, n = 0.0, 0.0, 0
@@ -657,7 +697,7 @@ def run_decode(args, local):
     gbs = compulsory / (ms * 1e-3) / 1e9
     per = {n: {"launches": c, "avg_ms": round(t / max(c, 1), 5)} for n, (t, c) in prof.items() if c}
     return {
-        "metric": "sparse MLA decode tokens/s (one new position per sequence, absorbed form)",
+        "metric": DECODE_METRIC,
         "value": round(B / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; no checkpoint)",
@@ -680,9 +720,33 @@ def run_decode(args, local):
     }
 
 
+def run_reference_decode(args):
+    """The oracle on decode units: each step is one (sequence, head) unit;
+    a token needs H of them, so tokens/s = 1 / (H x mean unit time)."""
+    B, T = args.B or 64, args.T or 32768
+    H, k = args.H or 128, args.topk or 2048
+    x = synth.make_decode_inputs(B, T, H, k, seed=11)
+    rng = np.random.default_rng(11)
+    for _ in range(args.warmup):
+        oracle_decode_unit(x, rng)
+    tot = sum(oracle_decode_unit(x, rng) for _ in range(args.steps))
+    v = args.steps / (tot * H)
+    sample = (f"{args.steps} random (sequence, head) units of decode_B{B}_T{T} (fp64 oracle, 1 host thread); "
+              f"a token is H = {H} units")
+    return {"impl": "reference", "metric": DECODE_METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": f"decode_B{B}_T{T}", "B": B, "T": T, "H": H, "topk": k, "weights": "bf16"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
+    if args.mode == "decode":
+        return run_reference_decode(args)
     name, x = workload(args)
     rng = np.random.default_rng(11)
     # Each step is one sampled (query row, head) unit; about 0.2 s each at

@@ -112,3 +112,36 @@ def test_decode_selection_sets():
     for row in other:
         vals = sorted(row.tolist())
         assert len(set(vals)) == 16 and vals[-1] == 49 and vals[0] >= 0
+
+
+def test_decode_reference_unit_is_the_oracle_row_per_head():
+    # The decode reference arm times the oracle on (sequence, head) units laid
+    # out as a compact causal problem over the selected positions; its output
+    # must be the oracle's own row s = T-1 for that head, and the heads'
+    # shares of W_o must add up to the row's output.
+    import numpy as np
+    import oracle
+    x = synth.make_inputs(0, B=1, T=64, H=2, topk=16, seed=5)
+    s = x.T - 1
+    tk = x.topk_idx[0, s]
+    sel = torch.unique(tk[(tk >= 0) & (tk <= s)])
+    attn_full, out_full = oracle.prefill_rows(x, [s])
+    out_sum = np.zeros_like(out_full)
+    for h in range(x.H):
+        y = bench.decode_unit_problem(x.q[0, s, h], x.kv_latent[0], x.k_pe[0], x.W_kvb, x.W_o, sel, h, x.scale)
+        attn_y, out_y = oracle.prefill_rows(y, [y.T - 1])
+        assert np.array_equal(attn_y[0, 0], attn_full[0, h])
+        out_sum += out_y
+    assert np.allclose(out_sum, out_full, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_reference_arm_prints_the_decode_metric():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--mode", "decode", "--B", "2",
+                        "--T", "200", "--H", "2", "--topk", "24", "--steps", "2", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["metric"] == bench.DECODE_METRIC and d["config"]["workload"] == "decode_B2_T200"
