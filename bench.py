@@ -219,11 +219,12 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle sampling
 
-def oracle_unit(x, rng):
+def oracle_unit(x, rng, act_e4m3: bool = False):
     """One sampled unit of the workload for the CPU oracle: a random
     (query row, head) pair, its attention over the selected keys (with the
     up-projection of those keys for that head) and that head's share of the
-    output projection. Returns (seconds, algorithmic flops of the unit)."""
+    output projection; with act_e4m3 the oracle's dynamic e4m3 activations.
+    Returns (seconds, algorithmic flops of the unit)."""
     import oracle
     b = int(rng.integers(0, x.B))
     s = int(rng.integers(0, x.T))
@@ -235,10 +236,10 @@ def oracle_unit(x, rng):
         tk = x.topk_idx[b, s]
         n_sel = int(torch.unique(tk[(tk >= 0) & (tk <= s)]).numel())
     t0 = time.perf_counter()
-    a = oracle.attend_rows(x, [row], heads=[h])
+    a = oracle.attend_rows(x, [row], heads=[h], act_e4m3=act_e4m3)
     full = np.zeros((1, x.H * 128))
     full[0, h * 128:(h + 1) * 128] = a[0, 0]
-    oracle.project_rows(x, full)
+    oracle.project_rows(x, full, act_e4m3=act_e4m3)
     dt = time.perf_counter() - t0
     flops = 2.0 * 512 * 256 + n_sel * (2 * 192 + 2 * 128) + 2.0 * 128 * 7168
     return dt, flops
@@ -284,11 +285,11 @@ def oracle_decode_unit(x, rng):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(x, budget_s: float, seed: int = 7):
+def cpu_baseline(x, budget_s: float, seed: int = 7, act_e4m3: bool = False):
     rng = np.random.default_rng(seed)
     tot_t, tot_f, n = 0.0, 0.0, 0
     while tot_t < budget_s and n < 10000:
-        dt, fl = oracle_unit(x, rng)
+        dt, fl = oracle_unit(x, rng, act_e4m3)
         tot_t += dt
         tot_f += fl
         n += 1
@@ -491,7 +492,8 @@ def run_ours(args, rank, world, local):
         "pages_note": "the source pages give only shapes and parameter counts: no throughput numbers or hardware",
     }
     if world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = {k: v for k, v in cpu_baseline(x, args.cpu_seconds).items() if k != "seconds"}
+        result["cpu_baseline"] = {k: v for k, v in cpu_baseline(x, args.cpu_seconds, act_e4m3=bool(act)).items()
+                                  if k != "seconds"}
     return result
 
 
@@ -751,20 +753,24 @@ def run_reference(args, rank, world):
     rng = np.random.default_rng(11)
     # Each step is one sampled (query row, head) unit; about 0.2 s each at
     # this workload, so a default run stays within a few minutes.
+    act8 = args.act == "e4m3"
     for _ in range(args.warmup):
-        oracle_unit(x, rng)
+        oracle_unit(x, rng, act8)
     tot_t, tot_f = 0.0, 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_unit(x, rng)
+        dt, fl = oracle_unit(x, rng, act8)
         tot_t += dt
         tot_f += fl
     v = tot_f / tot_t / 1e12
-    sample = f"{args.steps} random (query row, head) units of {name} (fp64 oracle, 1 host thread)"
+    sample = (f"{args.steps} random (query row, head) units of {name} (fp64 oracle, 1 host thread"
+              + (", dynamic e4m3 activations)" if act8 else ")"))
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H,
-                                                    "topk": x.topk},
+                                                    "topk": x.topk,
+                                                    "weights": "e4m3 block-128" if x.fp8 else "bf16",
+                                                    "activations": "e4m3 dynamic 1x128" if act8 else "bf16"},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

@@ -145,3 +145,13 @@ def test_decode_reference_arm_prints_the_decode_metric():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["metric"] == bench.DECODE_METRIC and d["config"]["workload"] == "decode_B2_T200"
+
+
+def test_reference_arm_follows_the_activation_mode():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "4", "--act", "e4m3",
+                        "--B", "1", "--T", "256", "--H", "2", "--steps", "2", "--warmup", "0"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["activations"] == "e4m3 dynamic 1x128" and d["config"]["weights"] == "e4m3 block-128"
+    assert "e4m3 activations" in d["cpu_baseline"]["sample"] and d["value"] > 0
