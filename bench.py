@@ -766,7 +766,8 @@ def run_reference(args, rank, world):
               + (", dynamic e4m3 activations)" if act8 else ")"))
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "strong" if args.parallel == "heads" else "weak",
+            "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H,
                                                     "topk": x.topk,
                                                     "weights": "e4m3 block-128" if x.fp8 else "bf16",
