@@ -69,6 +69,9 @@ def parse_args(argv=None):
     p.add_argument("--selections", type=int, default=1,
                    help="decode: rotate through this many different top-k selections, one per step (a device "
                         "copy of the next selection precedes every timed step); 1 repeats the same selection")
+    p.add_argument("--path", choices=["auto", "dense", "absorbed"], default="auto",
+                   help="attention path: the library's per-group choice (auto), every row block-dense, or every "
+                        "row absorbed (needs top-k indices)")
     p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
                    help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
     args = p.parse_args(argv)
@@ -219,30 +222,89 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle sampling
 
-def oracle_unit(x, rng, act_e4m3: bool = False):
-    """One sampled unit of the workload for the CPU oracle: a random
-    (query row, head) pair, its attention over the selected keys (with the
-    up-projection of those keys for that head) and that head's share of the
-    output projection; with act_e4m3 the oracle's dynamic e4m3 activations.
-    Returns (seconds, algorithmic flops of the unit)."""
+def host_info() -> dict:
+    """The host's core count and CPU model (for the CPU-baseline fields)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count() or 1, "cpu_model": model}
+
+
+def selected_sets(x, rows):
+    """A_s of each flattened row b*T + s: the distinct selected keys t <= s."""
+    out = []
+    for r in rows:
+        b, s = divmod(int(r), x.T)
+        if x.topk_idx is None:
+            out.append(torch.arange(s + 1))
+        else:
+            tk = x.topk_idx[b, s].to(torch.int64)
+            out.append(torch.unique(tk[(tk >= 0) & (tk <= s)]))
+    return out
+
+
+def oracle_sample(x, rows, act_e4m3: bool = False, threads: int = 1):
+    """The oracle's whole block on a sample of query rows: the attention of
+    every head (the fp64 up-projection of the keys these rows select, the
+    masked softmax and the value mix) and then W_o on the full rows, with the
+    heads spread over `threads` host threads (oracle.prefill_rows_threaded).
+    Returns (seconds, algorithmic flops credited).
+
+    The credit follows the GPU line's work model restricted to what the sample
+    computes: every key the sample's rows select is up-projected once per
+    head (2*512*256 FLOP; the full problem up-projects each of its B*T keys
+    once, so the per-key cost is the same), each selected (row, key) pair
+    costs H*(2*192 + 2*128) FLOP, and each row's output projection
+    2*H*128*7168 FLOP."""
     import oracle
-    b = int(rng.integers(0, x.B))
-    s = int(rng.integers(0, x.T))
-    h = int(rng.integers(0, x.H))
-    row = b * x.T + s
-    if x.topk_idx is None:
-        n_sel = s + 1
-    else:
-        tk = x.topk_idx[b, s]
-        n_sel = int(torch.unique(tk[(tk >= 0) & (tk <= s)]).numel())
+    sets = selected_sets(x, rows)
+    keys = 0
+    for b in sorted({int(r) // x.T for r in rows}):
+        mine = [a for r, a in zip(rows, sets) if int(r) // x.T == b and a.numel()]
+        if mine:
+            keys += int(torch.unique(torch.cat(mine)).numel())
+    pairs = sum(int(a.numel()) for a in sets)
+    flops = (keys * x.H * 2.0 * 512 * 256 + pairs * x.H * (2 * 192 + 2 * 128)
+             + len(rows) * 2.0 * x.H * 128 * 7168)
     t0 = time.perf_counter()
-    a = oracle.attend_rows(x, [row], heads=[h], act_e4m3=act_e4m3)
-    full = np.zeros((1, x.H * 128))
-    full[0, h * 128:(h + 1) * 128] = a[0, 0]
-    oracle.project_rows(x, full, act_e4m3=act_e4m3)
-    dt = time.perf_counter() - t0
-    flops = 2.0 * 512 * 256 + n_sel * (2 * 192 + 2 * 128) + 2.0 * 128 * 7168
-    return dt, flops
+    oracle.prefill_rows_threaded(x, rows, act_e4m3=act_e4m3, n_threads=threads)
+    return time.perf_counter() - t0, flops
+
+
+def sample_rows_cpu(x, rng, n: int):
+    """n random flattened rows (b*T + s) for one CPU sample pass."""
+    return sorted({int(rng.integers(0, x.B)) * x.T + int(rng.integers(0, x.T)) for _ in range(n)})
+
+
+def cpu_baseline(x, budget_s: float, total_flops: float, seed: int = 7, act_e4m3: bool = False):
+    """The oracle timed on the host cores: passes over fresh random rows
+    (4 rows, every head, then W_o) until `budget_s` is spent."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    threads = oracle.host_threads()
+    tot_t, tot_f, n_rows, passes = 0.0, 0.0, 0, 0
+    while tot_t < budget_s and passes < 1000:
+        rows = sample_rows_cpu(x, rng, 4)
+        dt, fl = oracle_sample(x, rows, act_e4m3, threads)
+        tot_t += dt
+        tot_f += fl
+        n_rows += len(rows)
+        passes += 1
+    rate = tot_f / tot_t
+    return {"value": rate / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{passes} passes over 4 random query rows of {x.name} ({n_rows} rows): the fp64 oracle's "
+                      f"whole block for those rows (up-projection of the keys they select, attention of all "
+                      f"{x.H} heads, W_o), heads spread over {threads} host threads; {tot_t:.1f} s",
+            "gflops": round(rate / 1e9, 3), **host_info(),
+            "extrapolated_full_step_s": round(total_flops / rate, 1),
+            "extrapolation": "extrapolated: the workload's algorithmic FLOPs per step over the sample's rate",
+            "seconds": tot_t}
 
 
 DECODE_METRIC = "sparse MLA decode tokens/s (one new position per sequence, absorbed form)"
@@ -283,21 +345,6 @@ def oracle_decode_unit(x, rng):
     t0 = time.perf_counter()
     oracle.prefill_rows(y, [y.T - 1])
     return time.perf_counter() - t0
-
-
-def cpu_baseline(x, budget_s: float, seed: int = 7, act_e4m3: bool = False):
-    rng = np.random.default_rng(seed)
-    tot_t, tot_f, n = 0.0, 0.0, 0
-    while tot_t < budget_s and n < 10000:
-        dt, fl = oracle_unit(x, rng, act_e4m3)
-        tot_t += dt
-        tot_f += fl
-        n += 1
-    return {"value": tot_f / tot_t / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} random (query row, head) units of {x.name}: fp64 up-projection of the row's "
-                      f"selected keys for that head, masked softmax, value mix and the head's slice of W_o; "
-                      f"{tot_t:.1f} s on 1 host thread",
-            "seconds": tot_t}
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -347,7 +394,9 @@ def run_ours(args, rank, world, local):
     act = mla.MLA_ACT_E4M3_DYNAMIC if args.act == "e4m3" else mla.MLA_ACT_BF16
     if act and not x.fp8:
         raise SystemExit("--act e4m3 needs a workload with e4m3 weights (--config 4)")
-    dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8, act=act)
+    path = {"auto": mla.MLA_PATH_AUTO, "dense": mla.MLA_PATH_BLOCK_DENSE, "absorbed": mla.MLA_PATH_ABSORBED}[args.path]
+    dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8, path=path,
+                         act=act)
     ws_bytes = mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_PREFILL, x.topk_idx is not None)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = torch.empty(x.B, x.T, 7168, dtype=torch.bfloat16, device=dev)
@@ -356,7 +405,7 @@ def run_ours(args, rank, world, local):
     def step(st=None):
         mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g.get("W_kvb_scale"),
                         g.get("W_o_scale"), topk_idx=g.get("topk_idx"), scale=x.scale, out=out,
-                        workspace=ws, stream=st or stream, act=act)
+                        workspace=ws, stream=st or stream, path=path, act=act)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -410,7 +459,7 @@ def run_ours(args, rank, world, local):
     d2h = host_out.numel() * host_out.element_size()
     pipe = mla.PrefillPipeline(x.B, x.T, x.H, g["W_kvb"], g["W_o"], g.get("W_kvb_scale"), g.get("W_o_scale"),
                                topk=x.topk_idx.shape[-1] if x.topk_idx is not None else None, scale=x.scale,
-                               device=dev, act=act)
+                               device=dev, path=path, act=act)
     for _ in range(3):
         pipe.submit(host_in, host_out)
     pipe.synchronize()
@@ -468,6 +517,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
                    "weights": "e4m3 block-128" if x.fp8 else "bf16",
                    "activations": "e4m3 dynamic 1x128" if act else "bf16",
+                   "path": args.path,
                    "parallelism": f"independent sequences x{world}",
                    "l2": "no flush: every step reads > 600 MB, inputs larger than the 126 MB L2"},
         "queries_per_s": round(qps, 1),
@@ -492,8 +542,8 @@ def run_ours(args, rank, world, local):
         "pages_note": "the source pages give only shapes and parameter counts: no throughput numbers or hardware",
     }
     if world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = {k: v for k, v in cpu_baseline(x, args.cpu_seconds, act_e4m3=bool(act)).items()
-                                  if k != "seconds"}
+        result["cpu_baseline"] = {k: v for k, v in cpu_baseline(x, args.cpu_seconds, wm["flops"],
+                                                                 act_e4m3=bool(act)).items() if k != "seconds"}
     return result
 
 
@@ -749,21 +799,27 @@ def run_reference(args, rank, world):
         return None
     if args.mode == "decode":
         return run_reference_decode(args)
+    import oracle
     name, x = workload(args)
+    wm = work_model(x)
     rng = np.random.default_rng(11)
-    # Each step is one sampled (query row, head) unit; about 0.2 s each at
-    # this workload, so a default run stays within a few minutes.
+    threads = oracle.host_threads()
+    # Each step is one sample pass: 2 random query rows, the oracle's whole
+    # block for them (every head, then W_o), heads spread over the host
+    # threads; a few seconds each at this workload, so a default run stays
+    # within a few minutes.
     act8 = args.act == "e4m3"
     for _ in range(args.warmup):
-        oracle_unit(x, rng, act8)
+        oracle_sample(x, sample_rows_cpu(x, rng, 2), act8, threads)
     tot_t, tot_f = 0.0, 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_unit(x, rng, act8)
+        dt, fl = oracle_sample(x, sample_rows_cpu(x, rng, 2), act8, threads)
         tot_t += dt
         tot_f += fl
     v = tot_f / tot_t / 1e12
-    sample = (f"{args.steps} random (query row, head) units of {name} (fp64 oracle, 1 host thread"
-              + (", dynamic e4m3 activations)" if act8 else ")"))
+    sample = (f"{args.steps} passes over 2 random query rows of {name}: the fp64 oracle's whole block for those "
+              f"rows (up-projection of the keys they select, attention of all {x.H} heads, W_o), heads spread "
+              f"over {threads} host threads" + (", dynamic e4m3 activations" if act8 else ""))
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "strong" if args.parallel == "heads" else "weak",
@@ -772,7 +828,11 @@ def run_reference(args, rank, world):
                                                     "topk": x.topk,
                                                     "weights": "e4m3 block-128" if x.fp8 else "bf16",
                                                     "activations": "e4m3 dynamic 1x128" if act8 else "bf16"},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+                             "gflops": round(v * 1e3, 3), **host_info(),
+                             "extrapolated_full_step_s": round(wm["flops"] / (v * 1e12), 1),
+                             "extrapolation": "extrapolated: the workload's algorithmic FLOPs per step over the "
+                                              "sample's rate"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

@@ -136,13 +136,20 @@ int mla_kv_upproject(const mla_dims* dims, const void* kv_latent, const void* W_
  *   scale    : softmax scale applied to q.k, finite and > 0 (192^-0.5 for
  *              these models)
  *   attn_out : bf16 [B, T, H, 128]. A query with no surviving key gets 0.
- * Softmax in fp32 (exp2 form); P and V enter the PV product as bf16 (f16).
+ * Softmax in fp32 (exp2 form). On the block-dense path the softmax weights
+ * P and the up-projected values v enter the PV product as f16 (three more
+ * mantissa bits than bf16): every |v| must stay below 65504 (the f16
+ * range). A larger v (|v| >= 65520 rounds to infinity) is detected in the
+ * up-projection's epilogue and recorded as device error 301 (see
+ * mla_device_status); the attention rows that read it are then undefined.
+ * RMS-normalised latents with trained weights give |v| of order 10.
  * Two ways to the same result (dims->path):
  *   block-dense: up-project every key (k_nope_h, v_h = W_kvb rows applied to
  *     kv_latent), then per (query tile, 128-key block holding a selected key)
  *     scores, mask, softmax, value mix;
- *   absorbed (DeepSeek-V2 "Multi-Head Latent Attention", the decode form
- *     applied to prefill rows): per query row, q_nope of each head is
+ *   absorbed (the generation-time form of the DeepSeek-V3.2-Exp "Sparse
+ *     attention" page's Explanation, where a decoded token scores the cached
+ *     latent directly, applied to prefill rows): per query row, q_nope of each head is
  *     multiplied into W_kvb's k_nope rows (q_abs, 512 wide), scored against
  *     the row's selected latent rows [kv_latent | k_pe] only, the softmax
  *     weights mix the latent rows, and W_kvb's v rows map the 512-wide
@@ -175,9 +182,10 @@ int mla_prefill(const mla_dims* dims, const void* q, const void* kv_latent,
                 mla_stream_t stream);
 
 /* Decode: one new position per sequence against its cache (DeepSeek-V3.2-
- * Exp "Sparse attention" at generation time, where the pages score the
- * cached latent directly: the absorbed form of DeepSeek-V2 "Multi-Head
- * Latent Attention"). Equals row s = T-1 of mla_prefill for a sequence whose
+ * Exp "Sparse attention" page, Explanation: at generation time a single
+ * decoded token scores the cached latent directly, i.e. the absorbed form
+ * with W_UK folded into the query and W_UV applied after the value mix).
+ * Equals row s = T-1 of mla_prefill for a sequence whose
  * first T-1 positions are the cache, up to rounding.
  *   dims     : B sequences, T = cache length including the new position
  *              (the query sits at s = T-1), H, topk, wdtype; path ignored
@@ -247,10 +255,35 @@ int mla_quantize_act(const void* x, int rows, int cols, void* codes, float* scal
 const char* mla_status_str(int status);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device. *device_error receives 0 (none) or the code a kernel
- * recorded (1xx: pipeline wait timed out; 2xx: bad launch geometry). Returns
- * MLA_ERR_CUDA if synchronisation fails, else MLA_OK. */
+ * current device. *device_error receives 0 (none) or the first code a
+ * kernel recorded: 1xx a pipeline wait timed out (101 TMA load, 102
+ * tensor-core commit, 103 consumer release, 104 epilogue, 105 softmax
+ * hand-off); 201 bad launch geometry; 301 an up-projected value v exceeded
+ * the f16 range (|v| >= 65520) on the attention path (see mla_attend).
+ * Returns MLA_ERR_CUDA if synchronisation fails, else MLA_OK. */
 int mla_device_status(mla_stream_t stream, int* device_error);
+
+/* Failure detection. Every on-chip wait of the kernels (mbarrier waits on
+ * TMA loads, tensor-core commits and hand-offs between warps) gives up after
+ * a time limit, records a 1xx code in the device error word, lets its
+ * in-flight copies and tensor-core work land (again bounded), releases its
+ * tensor memory and returns, so that a lost arrival ends as an error status
+ * instead of a hung GPU.
+ * mla_set_wait_timeout_ns sets that limit, in nanoseconds of the GPU's
+ * global timer, for kernels launched afterwards on the current device (0
+ * restores the default of 1 s). Synchronous with the host (a copy to a
+ * device variable); call it between launches, not during stream capture.
+ * Returns MLA_ERR_CUDA if no device is usable. */
+int mla_set_wait_timeout_ns(unsigned long long ns);
+
+/* Test hook for the failure path above, off by default: while on (on != 0)
+ * the producer warp of the block-dense attention kernel issues none of its
+ * loads on the current device, so that the kernel's waits for them (and for
+ * the tensor-core work that would follow) run into the time limit. The
+ * kernel then records a 1xx code and exits cleanly; its output is
+ * undefined. Nothing faults or hangs: every wait is bounded. Synchronous
+ * like mla_set_wait_timeout_ns; switch it off again before normal use. */
+int mla_test_withhold_attention_loads(int on);
 
 /* Per-kernel device timing (CUDA events on the launching stream).
  * mla_profile_begin() starts recording events around every launch made by

@@ -193,6 +193,41 @@ def prefill_rows(x, rows, **dims):
     return attn, out
 
 
+def host_threads() -> int:
+    """Threads the *_threaded helpers use by default (the host's cores, at most 32)."""
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def attend_rows_threaded(x, rows, heads=None, act_e4m3=False, n_threads=None) -> np.ndarray:
+    """attend_rows with the heads spread over host threads.
+
+    The oracle computes every head on its own (each call up-projects the keys
+    its heads need), so a call's heads can be split into shards that run at
+    once; ctypes releases the GIL while the C++ code runs. Each thread runs
+    the same plain single-threaded function on its shard and the shards are
+    put back in head order, so the result equals one call bit for bit."""
+    hs = list(range(int(x.H))) if heads is None else list(heads)
+    rows = list(rows)
+    n = max(1, min(n_threads or host_threads(), len(hs)))
+    shards = [hs[i::n] for i in range(n)]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(n) as ex:
+        parts = list(ex.map(lambda sh: attend_rows(x, rows, heads=sh, act_e4m3=act_e4m3), shards))
+    out = np.zeros((len(rows), len(hs), 128), dtype=np.float64)
+    for i in range(n):
+        out[:, i::n] = parts[i]
+    return out
+
+
+def prefill_rows_threaded(x, rows, act_e4m3=False, n_threads=None):
+    """prefill_rows with the attention's heads spread over host threads and
+    the output projection run once on the assembled rows (equal to
+    prefill_rows bit for bit)."""
+    attn = attend_rows_threaded(x, rows, act_e4m3=act_e4m3, n_threads=n_threads)
+    out = project_rows(x, attn.reshape(attn.shape[0], -1), act_e4m3=act_e4m3)
+    return attn, out
+
+
 def bf16_to_double(bits: int) -> float:
     return _load().mlao_bf16_to_double(int(bits) & 0xFFFF)
 

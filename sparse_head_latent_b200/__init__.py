@@ -34,6 +34,8 @@ from .mla import (  # noqa: F401
     mla_profile_begin,
     mla_profile_end,
     mla_quantize_act,
+    mla_set_wait_timeout_ns,
     mla_status_str,
+    mla_test_withhold_attention_loads,
     mla_workspace_bytes,
 )

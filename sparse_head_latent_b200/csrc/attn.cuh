@@ -186,7 +186,7 @@ sparse_mla_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   const Abort ab{abort_word, p.err};
 
   if (warp == 0) {
-    if (lane == 0 && n > 0) {
+    if (lane == 0 && n > 0 && *reinterpret_cast<volatile int*>(&g_mla_withhold_attn_loads) == 0) {
       // ---------------- TMA producer (this CTA's halves; completion is
       // counted on the leader's barriers, which expect both CTAs' bytes)
       int nk = 0, nv = 0;

@@ -4,8 +4,9 @@
 // The block-dense kernel (attn.cuh) up-projects every key and visits every
 // 128-key block that holds a selected key; for a row s with s + 1 >> k
 // nearly all of that work is masked away. Here each row attends only its
-// selected keys, in the latent space (DeepSeek-V2 "Multi-Head Latent
-// Attention", absorbed form; the same per-head weights as the prefill path):
+// selected keys, in the latent space: the form the DeepSeek-V3.2-Exp "Sparse
+// attention" page's Explanation names for a decoded token, which scores the
+// cached latent directly (same per-head weights as the prefill path):
 //   q_abs[h] = q_nope[h] . W_UK[h]            (absorb GEMM, before this kernel)
 //   z_t      = [q_abs[h] | q_pe[h]] . [c_t | k_pe_t]     t in A_s, 576 wide
 //   o_lat[h] = sum_t softmax(z * scale)_t c_t            (this kernel)
@@ -262,7 +263,7 @@ absorbed_attn_kernel(const AbsParams p) {
           const uint64_t now = global_timer_ns();
           if (t_idle == 0) {
             t_idle = now;
-          } else if (now - t_idle > kWaitTimeoutNs || ab.raised()) {
+          } else if (now - t_idle > wait_timeout_ns() || ab.raised()) {
             if (!ab.raised()) ab.raise(kErrWaitSoftmax);
             ok = false;
           }

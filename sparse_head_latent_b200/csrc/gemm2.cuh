@@ -212,6 +212,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const int q = warp & 3;
     uint8_t* bufs = epi + (warp - 2) * 2 * Cfg::EPI_BUF;
     int t = 0, nbuf = 0;
+    float vmax = 0.f;  // largest |value| stored as f16 (V_F16)
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
       const int bi = tile / (num_m * num_n);
       int mt, nt;
@@ -243,6 +244,8 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const float* f1 = reinterpret_cast<const float*>(r1) + 8 * j;
           uint4 v0, v1;
           if (f16) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vmax = max3(vmax, fabsf(f0[i]), fabsf(f1[i]));
             v0 = make_uint4(pack_f16x2(f0[0], f0[1]), pack_f16x2(f0[2], f0[3]), pack_f16x2(f0[4], f0[5]),
                             pack_f16x2(f0[6], f0[7]));
             v1 = make_uint4(pack_f16x2(f1[0], f1[1]), pack_f16x2(f1[2], f1[3]), pack_f16x2(f1[4], f1[5]),
@@ -269,6 +272,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       if (lane == 0) mbar_arrive_remote(mapa_shared(acce0 + 8 * a, 0));
     }
     if (lane == 0) bulk_wait_group<0>();
+    if (Cfg::V_F16 && __any_sync(0xffffffffu, vmax >= kF16Overflow) && lane == 0) atomicCAS(err, 0, kErrRangeF16);
   }
 
   tc_fence_before();

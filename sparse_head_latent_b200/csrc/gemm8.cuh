@@ -220,6 +220,7 @@ gemm_e4m3_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + hh * CW;
     int pc = 0, nbuf = 0;
     bool ok = true;
+    float vmax = 0.f;  // largest |value| stored as f16 (V_F16)
     for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
       int mt, nt;
       grouped_tile(tile, num_m, num_n, Cfg::GROUP_M, mt, nt);
@@ -288,12 +289,15 @@ gemm_e4m3_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         for (int j = 0; j < 8; ++j) {
           const float* v = acc + 64 * c + 8 * j;
           uint4 u;
-          if (f16)
+          if (f16) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) vmax = max3(vmax, fabsf(v[i]), fabsf(v[i + 1]));
             u = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
                            pack_f16x2(v[6], v[7]));
-          else
+          } else {
             u = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                            pack_bf16x2(v[6], v[7]));
+          }
           *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = u;
         }
         fence_proxy_async_smem();
@@ -306,6 +310,7 @@ gemm_e4m3_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
     }
     if (lane == 0) bulk_wait_group<0>();
+    if (Cfg::V_F16 && __any_sync(0xffffffffu, vmax >= kF16Overflow) && lane == 0) atomicCAS(err, 0, kErrRangeF16);
   }
 
   tc_fence_before();

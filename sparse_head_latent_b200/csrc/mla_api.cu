@@ -1063,6 +1063,20 @@ int mla_device_status(mla_stream_t stream, int* device_error) {
   return MLA_OK;
 }
 
+int mla_set_wait_timeout_ns(unsigned long long ns) {
+  const unsigned long long v = ns == 0 ? mla::kWaitTimeoutNs : ns;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  return cudaMemcpyToSymbol(mla::g_mla_wait_timeout_ns, &v, sizeof v) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_test_withhold_attention_loads(int on) {
+  const int v = on != 0 ? 1 : 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  return cudaMemcpyToSymbol(mla::g_mla_withhold_attn_loads, &v, sizeof v) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_profile_begin(void) {
   for (auto& r : t_prof.recs) {
     t_prof.pool.push_back(r.start);

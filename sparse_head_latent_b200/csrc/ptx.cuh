@@ -18,11 +18,29 @@ enum : int {
   kErrWaitEpilogue = 104, // a wait for the epilogue timed out
   kErrWaitSoftmax = 105,  // a wait for the softmax warps timed out
   kErrGeometry = 201,     // launch geometry does not match the kernel's assumptions
+  kErrRangeF16 = 301,     // an up-projected v exceeded the f16 range of the attention path
 };
 
+// Magnitude from which fp32 -> f16 rounding (nearest even) gives infinity:
+// halfway between the largest finite f16 (65504) and 2^16.
+constexpr float kF16Overflow = 65520.f;
+
 // A pipeline wait gives up after this long (ns of %globaltimer). No wait in
-// these kernels legitimately lasts more than microseconds.
+// these kernels legitimately lasts more than microseconds. The default is
+// kWaitTimeoutNs; the host may lower it per device (mla_set_wait_timeout_ns)
+// for kernels launched afterwards.
 constexpr uint64_t kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s
+__device__ unsigned long long g_mla_wait_timeout_ns = kWaitTimeoutNs;
+
+__device__ __forceinline__ uint64_t wait_timeout_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_mla_wait_timeout_ns);
+}
+
+// Test hook, 0 in normal use: when set, the producer of the block-dense
+// attention kernel issues none of its loads, so the kernel's bounded waits
+// expire; it exercises the abort path (error word, clean exit) without any
+// fault.
+__device__ int g_mla_withhold_attn_loads = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -102,10 +120,40 @@ struct Abort {
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = wait_timeout_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (ab.raised()) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > limit) {
+      ab.raise(code);
+      return false;
+    }
+  }
+}
+
+// mbar_wait with cluster-scope acquire: for a phase completed by arrivals
+// that release shared-memory writes of the peer CTA (cluster-scope release),
+// which this thread then hands to the tensor core.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const Abort& ab, int code) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = wait_timeout_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (ab.raised()) return false;
+    if (global_timer_ns() - t0 > limit) {
       ab.raise(code);
       return false;
     }
@@ -123,8 +171,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const A
 // Bounded wait used while draining after an abort: never records an error.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
+  const uint64_t limit = wait_timeout_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    if (global_timer_ns() - t0 > limit) return false;
   }
   return true;
 }

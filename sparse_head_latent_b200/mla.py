@@ -58,6 +58,8 @@ SIGNATURES = {
     "mla_quantize_act": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP]),
     "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int)]),
+    "mla_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
+    "mla_test_withhold_attention_loads": (ctypes.c_int, [ctypes.c_int]),
     "mla_profile_begin": (ctypes.c_int, []),
     "mla_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
 }
@@ -170,13 +172,13 @@ MLA_STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def mla_attend_static(q, kv_latent, k_pe, W_kvb, W_kvb_scale=None, topk_idx=None, scale=192 ** -0.5,
-                      attn_out=None, stream=None):
+                      attn_out=None, stream=None, path=MLA_PATH_AUTO, act=MLA_ACT_BF16):
     """mla_attend with the library's built-in scratch instead of a workspace,
     for callers that cannot allocate device memory; problems whose scratch
     exceeds MLA_STATIC_SCRATCH_BYTES are rejected (MlaError, status 8)."""
     B, T, H, _ = q.shape
     topk = 0 if topk_idx is None else topk_idx.shape[-1]
-    dims = make_dims(B, T, H, topk, _wtype(W_kvb))
+    dims = make_dims(B, T, H, topk, _wtype(W_kvb), path, act)
     if topk_idx is not None and topk_idx.dtype != torch.int32:
         raise ValueError("topk_idx must be int32")
     if attn_out is None:
@@ -267,6 +269,18 @@ def mla_device_status(stream=None) -> int:
     return v.value
 
 
+def mla_set_wait_timeout_ns(ns: int):
+    """Time limit of the kernels' on-chip waits on the current device, for
+    launches from now on (0 restores the 1 s default)."""
+    _check("mla_set_wait_timeout_ns", load_library().mla_set_wait_timeout_ns(int(ns)))
+
+
+def mla_test_withhold_attention_loads(on: bool):
+    """Test hook: while on, the block-dense attention kernel issues no loads
+    and its bounded waits expire (error word 1xx, clean exit)."""
+    _check("mla_test_withhold_attention_loads", load_library().mla_test_withhold_attention_loads(1 if on else 0))
+
+
 def mla_profile_begin():
     _check("mla_profile_begin", load_library().mla_profile_begin())
 
@@ -292,7 +306,7 @@ class PrefillPipeline:
     _INPUTS = ("q", "kv_latent", "k_pe", "topk_idx")
 
     def __init__(self, B, T, H, W_kvb, W_o, W_kvb_scale=None, W_o_scale=None, topk=None,
-                 scale=192 ** -0.5, device=None, act=MLA_ACT_BF16):
+                 scale=192 ** -0.5, device=None, path=MLA_PATH_AUTO, act=MLA_ACT_BF16):
         dev = torch.device(device) if device is not None else W_o.device
         self.dev, self.scale = dev, float(scale)
         self.w = dict(W_kvb=W_kvb, W_o=W_o, W_kvb_scale=W_kvb_scale, W_o_scale=W_o_scale)
@@ -303,8 +317,8 @@ class PrefillPipeline:
         self.slots = [{k: torch.empty(s, dtype=d, device=dev) for k, (s, d) in shapes.items()} for _ in range(2)]
         for sl in self.slots:
             sl["out"] = torch.empty(B, T, D_MODEL, dtype=torch.bfloat16, device=dev)
-        self.act = int(act)
-        dims = make_dims(B, T, H, 0 if topk is None else topk, _wtype(W_kvb), act=self.act)
+        self.act, self.path = int(act), int(path)
+        dims = make_dims(B, T, H, 0 if topk is None else topk, _wtype(W_kvb), path=self.path, act=self.act)
         self.ws = torch.empty(max(1, mla_workspace_bytes(dims, MLA_ENTRY_PREFILL, topk is not None)),
                               dtype=torch.uint8, device=dev)
         self.h2d, self.comp, self.d2h = (torch.cuda.Stream(dev) for _ in range(3))
@@ -330,7 +344,7 @@ class PrefillPipeline:
             self.comp.wait_event(self.ev_out[k])  # the previous output of this slot has been copied out
         mla_prefill(sl["q"], sl["kv_latent"], sl["k_pe"], self.w["W_kvb"], self.w["W_o"], self.w["W_kvb_scale"],
                     self.w["W_o_scale"], topk_idx=sl.get("topk_idx"), scale=self.scale, out=sl["out"],
-                    workspace=self.ws, stream=self.comp, act=self.act)
+                    workspace=self.ws, stream=self.comp, path=self.path, act=self.act)
         self.ev_done[k].record(self.comp)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.ev_done[k])

@@ -203,3 +203,28 @@ def test_workspace_sizes_decode(lib):
     d = MlaDims(B, 1000, H, 128, 64, 128, 512, 7168, k, 0, 0, 0)
     assert mla.mla_workspace_bytes(d, mla.MLA_ENTRY_DECODE, True) == (
         2 * up(B * H * 512 * 2) + up(B * kpad * 4) + up(B * 4) + up(B * H * 128 * 2))
+
+
+def test_static_scratch_limit_agrees_with_the_library(lib):
+    # MLA_STATIC_SCRATCH_BYTES is written out in both include/mla.h and the
+    # Python binding; the library's own size check must draw the line exactly
+    # there: a problem whose attend workspace is exactly that size passes the
+    # size check, one 1 KB larger is rejected with status 8 before any
+    # device work. (Host-only: on a machine with a GPU the accepted case
+    # would go on to launch kernels on the placeholder pointers, so it is
+    # skipped there.)
+    import torch
+    from sparse_head_latent_b200.mla import MLA_STATIC_SCRATCH_BYTES
+    header = open(HEADER).read()
+    m = re.search(r"#define MLA_STATIC_SCRATCH_BYTES \((\d+)u << (\d+)\)", header)
+    assert m and int(m.group(1)) << int(m.group(2)) == MLA_STATIC_SCRATCH_BYTES
+    fits = mla.make_dims(1, 32768, 2, 0, False)  # up-projected kv: 32768 x 2 x 512 B = 32 MiB
+    over = mla.make_dims(1, 32769, 2, 0, False)
+    assert mla.mla_workspace_bytes(fits, mla.MLA_ENTRY_ATTEND, False) == MLA_STATIC_SCRATCH_BYTES
+    assert mla.mla_workspace_bytes(over, mla.MLA_ENTRY_ATTEND, False) > MLA_STATIC_SCRATCH_BYTES
+    call = lambda d: lib.mla_attend_static(ctypes.byref(d), 16, 16, 16, 16, None, None,  # noqa: E731
+                                           ctypes.c_float(0.07), 16, None)
+    assert call(over) == 8
+    if torch.cuda.is_available():
+        pytest.skip("the accepted case would launch kernels on placeholder pointers")
+    assert call(fits) not in (0, 8)  # passes the size check, then finds no usable device

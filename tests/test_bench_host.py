@@ -78,7 +78,9 @@ def test_reference_arm_prints_one_line_on_rank_zero_only():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["nproc"] >= cb["cores"] and cb["cpu_model"]
+    assert cb["extrapolated_full_step_s"] > 0 and "extrapolated" in cb["extrapolation"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0
     env["RANK"], env["WORLD_SIZE"] = "1", "2"
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "0", "--steps", "3"],
@@ -88,9 +90,25 @@ def test_reference_arm_prints_one_line_on_rank_zero_only():
 
 def test_cpu_baseline_sample_is_bounded():
     x = synth.make_inputs(0)
-    d = bench.cpu_baseline(x, 0.5)
-    assert d["kind"] == "oracle" and d["cores"] == 1 and d["value"] > 0
+    d = bench.cpu_baseline(x, 0.5, 2.2e9)
+    assert d["kind"] == "oracle" and d["cores"] >= 1 and d["value"] > 0
     assert d["seconds"] < 5
+    assert d["nproc"] >= 1 and d["extrapolated_full_step_s"] > 0
+
+
+def test_oracle_sample_credits_the_work_model():
+    # Two rows of one sequence: every key either selects is up-projected once
+    # per head, every selected pair costs H * 640 FLOP, every row's W_o
+    # 2 * H * 128 * 7168 FLOP (the GPU line's work model).
+    x = synth.make_inputs(0, B=1, T=64, H=2, topk=8, seed=9)
+    rows = [10, 63]
+    sets = bench.selected_sets(x, rows)
+    keys = len(set(sets[0].tolist()) | set(sets[1].tolist()))
+    pairs = len(sets[0]) + len(sets[1])
+    assert len(sets[0]) == 8 and len(sets[1]) == 8  # s always selected, plus 7 distinct earlier keys
+    dt, fl = bench.oracle_sample(x, rows, threads=2)
+    assert dt > 0
+    assert fl == keys * 2 * 2 * 512 * 256 + pairs * 2 * 640 + 2 * 2 * 2 * 128 * 7168
 
 
 def test_step_defaults_per_mode():

@@ -97,6 +97,34 @@ def test_output_projection_matches_oracle(rows, H, fp8):
     assert_close(out.float().cpu().numpy(), ref, "out")
 
 
+def _dequant_bf16(codes, scale):
+    """bf16(e4m3(code) * block scale), the fp32 product rounded to nearest even."""
+    R, C = codes.shape
+    f = codes.view(torch.float8_e4m3fn).to(torch.float32).view(R // 128, 128, C // 128, 128)
+    return (f * scale[:, None, :, None]).view(R, C).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("stage", ["kv_upproject", "out_project"])
+def test_fp8_weight_gemms_equal_the_bf16_gemm_on_the_dequantised_weight(stage):
+    # With bf16 activations the e4m3 weight tiles are converted on chip
+    # (code exactly, times its 128 x 128 block scale in fp32, rounded to
+    # bf16) and fed to the bf16 tensor-core GEMM; the bf16 GEMM on the weight
+    # dequantised the same way on the host must give the same bits. Several
+    # row tiles (ragged), column tiles and 128-deep K blocks.
+    x = synth.make_inputs(0, B=1, T=600, H=4, topk=None, seed=36, fp8=True)
+    g = _dev(x)
+    if stage == "kv_upproject":
+        got = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"], g["W_kvb_scale"])
+        ref = mla.mla_kv_upproject(g["kv_latent"], _dequant_bf16(x.W_kvb, x.W_kvb_scale).cuda())
+    else:
+        gen = torch.Generator().manual_seed(37)
+        attn = (0.05 * torch.randn(x.T, x.H * 128, generator=gen)).to(torch.bfloat16).cuda()
+        got = mla.mla_out_project(attn, g["W_o"], g["W_o_scale"])
+        ref = mla.mla_out_project(attn, _dequant_bf16(x.W_o, x.W_o_scale).cuda())
+    _no_device_error()
+    assert torch.equal(got, ref)
+
+
 # ---------------------------------------------------------------- attention
 
 ATTEND_CASES = {
@@ -123,6 +151,25 @@ def test_attend_matches_oracle(case):
     attn = _attend(x, g)
     _no_device_error()
     ref = oracle.attend_rows(x, range(x.B * x.T))
+    assert_close(attn.float().cpu().numpy().reshape(ref.shape), ref, case)
+
+
+# The full head count of the headline workload, compared in full: the head-
+# group scheduler (groups of 8 heads, heaviest tile groups first) and the
+# tile-group logic at H = 128, on a sparse case and a ragged causal one.
+FULL_HEAD_CASES = {
+    "h128_sparse": dict(B=1, T=1024, H=128, topk=256),
+    "h128_ragged_causal": dict(B=2, T=700, H=128, topk=None),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FULL_HEAD_CASES))
+def test_attend_all_128_heads_matches_oracle(case):
+    x = synth.make_inputs(0, seed=35, **FULL_HEAD_CASES[case])
+    g = _dev(x)
+    attn = _attend(x, g)
+    _no_device_error()
+    ref = oracle.attend_rows_threaded(x, range(x.B * x.T))
     assert_close(attn.float().cpu().numpy().reshape(ref.shape), ref, case)
 
 

@@ -434,3 +434,17 @@ def test_act_e4m3_block_equals_dense_restatement(fp8):
     _, out_bf16 = oracle.prefill_rows(x, _all_rows(x))
     d = np.linalg.norm(out - out_bf16) / np.linalg.norm(out_bf16)
     assert 1e-3 < d < 0.1   # e4m3 activations move the output by about a percent
+
+
+def test_threaded_oracle_equals_the_plain_calls_bit_for_bit():
+    # The tests and the benchmark's CPU leg spread the oracle's heads over
+    # host threads; the shards must reassemble to exactly the plain result.
+    for cfg, fp8, act in ((0, False, False), (4, True, True)):
+        x = synth.make_inputs(cfg, B=2, T=200, H=5, topk=24, seed=91, fp8=fp8)
+        rows = [0, 17, 199, 200, 333, 399]
+        a1, o1 = oracle.prefill_rows(x, rows, act_e4m3=act)
+        a2, o2 = oracle.prefill_rows_threaded(x, rows, act_e4m3=act, n_threads=3)
+        assert np.array_equal(a1, a2) and np.array_equal(o1, o2)
+        h = [4, 0, 2]
+        assert np.array_equal(oracle.attend_rows(x, rows, heads=h), oracle.attend_rows_threaded(x, rows, heads=h,
+                                                                                              n_threads=2))

@@ -22,10 +22,10 @@ from sparse_head_latent_b200.mla import MLA_STATIC_SCRATCH_BYTES, make_dims
 MAX_ABS, REL_L2 = 2e-2, 5e-3  # the tolerance every GPU parity test uses
 
 
-def _static_via_abi(lib, x, g):
+def _static_via_abi(lib, x, g, path=mla.MLA_PATH_AUTO, act=mla.MLA_ACT_BF16):
     """One mla_attend_static call through the C ABI; returns (status, attn)."""
     tk = g.get("topk_idx")
-    dims = make_dims(x.B, x.T, x.H, 0 if tk is None else tk.shape[-1], x.fp8)
+    dims = make_dims(x.B, x.T, x.H, 0 if tk is None else tk.shape[-1], x.fp8, path, act)
     attn = torch.full((x.B, x.T, x.H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
     sc = g.get("W_kvb_scale")
     rc = lib.mla_attend_static(ctypes.byref(dims), g["q"].data_ptr(), g["kv_latent"].data_ptr(),
@@ -47,18 +47,29 @@ def _close(got, ref):
 @pytest.mark.gpu
 def test_static_scratch_entry_matches_workspace_entry_on_two_calls_in_a_row():
     lib = mla.load_library()
-    # Two different problems back to back: the second call finds the first
-    # call's contents in the shared array and must not depend on them.
-    cases = [synth.make_inputs(0, B=2, T=300, H=4, topk=40, seed=71),
-             synth.make_inputs(0, B=1, T=200, H=2, topk=None, seed=72)]
-    for x in cases:
+    # Different problems back to back: each call finds the previous call's
+    # contents in the shared array and must not depend on them. The cases
+    # place every scratch region in the array at least once: up-projected kv,
+    # bitmap and block lists (block-dense), the per-row key lists, q_abs and
+    # o_lat of the absorbed rows, the dequantised e4m3 W_kvb, and the
+    # quantized latent of the e4m3-activation mode.
+    A, D = mla.MLA_PATH_ABSORBED, mla.MLA_PATH_BLOCK_DENSE
+    cases = [(synth.make_inputs(0, B=2, T=300, H=4, topk=40, seed=71), mla.MLA_PATH_AUTO, 0),
+             (synth.make_inputs(0, B=1, T=1200, H=4, topk=40, seed=73), A, 0),
+             (synth.make_inputs(0, B=1, T=200, H=2, topk=None, seed=72), D, 0),
+             (synth.make_inputs(0, B=1, T=1200, H=4, topk=40, seed=73), A, 0),
+             (synth.make_inputs(0, B=2, T=300, H=4, topk=40, seed=74, fp8=True), D, 0),
+             (synth.make_inputs(0, B=1, T=300, H=4, topk=40, seed=75, fp8=True), D, mla.MLA_ACT_E4M3_DYNAMIC)]
+    for x, path, act in cases:
         g = {k: v.cuda() for k, v in x.tensors().items()}
-        rc, got = _static_via_abi(lib, x, g)
+        rc, got = _static_via_abi(lib, x, g, path, act)
         assert rc == 0, mla.mla_status_str(rc)
         ref = mla.mla_attend(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g.get("W_kvb_scale"),
-                             topk_idx=g.get("topk_idx"), scale=x.scale)
+                             topk_idx=g.get("topk_idx"), scale=x.scale, path=path, act=act)
         assert mla.mla_device_status() == 0
         _close(got, ref)
+        # the same kernels on the same inputs: bit for bit
+        assert torch.equal(got, ref), (x.T, path, act)
 
 
 def test_static_scratch_entry_rejects_problems_beyond_its_scratch():
