@@ -40,7 +40,7 @@ import synth  # noqa: E402
 METRIC = "sparse MLA prefill TFLOP/s and queries/s (T=4096,H=128,top-k 2048); % of bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "gemm_m64.cuh", "quant.cuh", "attn.cuh", "attn_abs.cuh",
+KERNEL_SOURCES = ("ptx.cuh", "gemm2.cuh", "gemm8.cuh", "gemm_w8t.cuh", "gemm_m64.cuh", "quant.cuh", "attn.cuh", "attn_abs.cuh",
                   "prepass.cuh",
                   "dequant.cuh", "mla_api.cu")
 
@@ -74,6 +74,9 @@ def parse_args(argv=None):
                         "row absorbed (needs top-k indices)")
     p.add_argument("--act", choices=["bf16", "e4m3"], default="bf16",
                    help="activations entering the projections (e4m3: dynamic per-token, needs e4m3 weights)")
+    p.add_argument("--e4m3-weights", choices=["dequant", "onchip"], default="dequant",
+                   help="e4m3 weights with bf16 activations: a dequantised bf16 copy per call (default), or "
+                        "converted on chip inside the projection GEMMs")
     args = p.parse_args(argv)
     if args.steps is None:
         args.steps = 2000 if args.mode == "decode" and args.impl == "ours" else 200
@@ -395,6 +398,7 @@ def run_ours(args, rank, world, local):
     if act and not x.fp8:
         raise SystemExit("--act e4m3 needs a workload with e4m3 weights (--config 4)")
     path = {"auto": mla.MLA_PATH_AUTO, "dense": mla.MLA_PATH_BLOCK_DENSE, "absorbed": mla.MLA_PATH_ABSORBED}[args.path]
+    mla.mla_set_e4m3_weight_conversion(args.e4m3_weights == "onchip")
     dims = mla.make_dims(x.B, x.T, x.H, x.topk_idx.shape[-1] if x.topk_idx is not None else 0, x.fp8, path=path,
                          act=act)
     ws_bytes = mla.mla_workspace_bytes(dims, mla.MLA_ENTRY_PREFILL, x.topk_idx is not None)
@@ -517,6 +521,8 @@ def run_ours(args, rank, world, local):
         "config": {"workload": name, "B": x.B, "T": x.T, "H": x.H, "topk": x.topk,
                    "weights": "e4m3 block-128" if x.fp8 else "bf16",
                    "activations": "e4m3 dynamic 1x128" if act else "bf16",
+                   **({"e4m3_weights": "converted on chip" if args.e4m3_weights == "onchip" else "dequantised copy"}
+                      if x.fp8 and not act else {}),
                    "path": args.path,
                    "parallelism": f"independent sequences x{world}",
                    "l2": "no flush: every step reads > 600 MB, inputs larger than the 126 MB L2"},

@@ -263,6 +263,26 @@ const char* mla_status_str(int status);
  * Returns MLA_ERR_CUDA if synchronisation fails, else MLA_OK. */
 int mla_device_status(mla_stream_t stream, int* device_error);
 
+/* How e4m3 weights (MLA_W_E4M3_BLOCK128) meet bf16 activations (MLA_ACT_BF16)
+ * in the projections, process-wide for calls made afterwards (Kimi K2 page,
+ * "Down projection": weights stored as e4m3 codes with one fp32 scale per
+ * 128 x 128 block; here each weight becomes bf16(code * scale), the fp32
+ * product rounded once, and meets the bf16 activations on the tensor cores).
+ *   onchip = 0 (default): each call dequantises W_kvb / W_o into a bf16 copy
+ *     in its workspace, then runs the bf16 GEMMs.
+ *   onchip = 1: the W_kvb and W_o GEMMs of prefill read the e4m3 codes and
+ *     their scales directly: converter warps turn each code tile into bf16
+ *     in tensor memory (the UMMA A operand of a transposed GEMM), so no copy
+ *     is written. Bit-identical to mode 0; measured slower on B200 at the
+ *     batched workload (B 16, T 1024, H 128): W_kvb 0.63 against 0.45 ms,
+ *     W_o 3.6 against 2.7 ms, because the conversion is repeated for every
+ *     token tile. The absorbed rows' GEMMs and mla_decode keep a bf16 copy of
+ *     W_kvb (and decode one of W_o) in both modes.
+ * mla_workspace_bytes() follows the mode in force when it is called: query
+ * it after switching. Host-only (no device work); returns MLA_ERR_SHAPE for
+ * an onchip value other than 0 or 1. */
+int mla_set_e4m3_weight_conversion(int onchip);
+
 /* Failure detection. Every on-chip wait of the kernels (mbarrier waits on
  * TMA loads, tensor-core commits and hand-offs between warps) gives up after
  * a time limit, records a 1xx code in the device error word, lets its

@@ -34,6 +34,7 @@ from .mla import (  # noqa: F401
     mla_profile_begin,
     mla_profile_end,
     mla_quantize_act,
+    mla_set_e4m3_weight_conversion,
     mla_set_wait_timeout_ns,
     mla_status_str,
     mla_test_withhold_attention_loads,

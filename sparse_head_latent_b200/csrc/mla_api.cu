@@ -17,6 +17,7 @@
 #include "attn_abs.cuh"
 #include "dequant.cuh"
 #include "gemm2.cuh"
+#include "gemm_w8t.cuh"
 #include "gemm8.cuh"
 #include "gemm_m64.cuh"
 #include "prepass.cuh"
@@ -33,7 +34,10 @@ using Gemm2Kvb = mla::Gemm2Cfg<false>;  // latent x W_kvb^T  (B stored [N, K])
 using Gemm2KvbAttn = mla::Gemm2Cfg<false, true>;  // same, v columns written as f16 for the attention
 using Gemm2Wo = mla::Gemm2Cfg<true>;    // attn x W_o         (B stored [K, N]); also q_nope x W_UK
 using Gemm2Unabs = mla::Gemm2Cfg<false, false, 128>;  // o_lat x W_UV^T (B stored [N, K], 128 wide)
-using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;  // attn x W_o with one row tile (decode): twice the pairs
+using Gemm2WoNarrow = mla::Gemm2Cfg<true, false, 128>;
+using GemmW8tKvb = mla::GemmW8tCfg<false, true>;            // latent x e4m3 W_kvb^T, weights converted on chip
+using GemmW8tKvbAttn = mla::GemmW8tCfg<false, true, true>;  // same, v columns written as f16 for the attention
+using GemmW8tWo = mla::GemmW8tCfg<true, false>;             // attn x e4m3 W_o, weights converted on chip  // attn x W_o with one row tile (decode): twice the pairs
 using GemmM64 = mla::GemmM64Cfg<64>;     // decode's output projection (stream-K), M <= 64
 using GemmM128 = mla::GemmM64Cfg<128>;   // and 64 < M <= 256 (128-row tiles)
 using GemmM64Abs = mla::GemmM64Cfg<64, true, true>;     // decode's q_nope x W_UK per head, bf16 out
@@ -52,6 +56,8 @@ struct DeviceState {
   int sms = 0;
   int pairs_kvb = 0;   // CTA pairs of the pair GEMMs that fit on the device at once
   int pairs_wo = 0;
+  int pairs_w8t_kvb = 0;  // CTA pairs of the e4m3-weight GEMMs with on-chip conversion
+  int pairs_w8t_wo = 0;
   int pairs_unabs = 0;
   int pairs_wo_narrow = 0;
   int pairs8_kvb = 0;  // CTA pairs of the e4m3 GEMMs
@@ -117,9 +123,17 @@ int device_state(DeviceState** out) {
       if (ok) {
         st.pairs_kvb = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Kvb>, Gemm2Kvb::SMEM_BYTES);
         st.pairs_wo = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Wo>, Gemm2Wo::SMEM_BYTES);
+        ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_w8t_kernel<GemmW8tKvb>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GemmW8tKvb::SMEM_BYTES) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_w8t_kernel<GemmW8tKvbAttn>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GemmW8tKvbAttn::SMEM_BYTES) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(mla::gemm_bf16_w8t_kernel<GemmW8tWo>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, GemmW8tWo::SMEM_BYTES) == cudaSuccess;
+        st.pairs_w8t_kvb = max_pairs(mla::gemm_bf16_w8t_kernel<GemmW8tKvb>, GemmW8tKvb::SMEM_BYTES, GemmW8tKvb::THREADS);
+        st.pairs_w8t_wo = max_pairs(mla::gemm_bf16_w8t_kernel<GemmW8tWo>, GemmW8tWo::SMEM_BYTES, GemmW8tWo::THREADS);
         st.pairs_unabs = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2Unabs>, Gemm2Unabs::SMEM_BYTES);
         st.pairs_wo_narrow = max_pairs(mla::gemm_bf16_tc2_kernel<Gemm2WoNarrow>, Gemm2WoNarrow::SMEM_BYTES);
-        ok = st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_unabs > 0 && st.pairs_wo_narrow > 0;
+        ok = ok && st.pairs_kvb > 0 && st.pairs_wo > 0 && st.pairs_w8t_kvb > 0 && st.pairs_w8t_wo > 0 && st.pairs_unabs > 0 && st.pairs_wo_narrow > 0;
       }
       ok = ok && cudaFuncSetAttribute(mla::gemm_e4m3_tc2_kernel<Gemm8Kvb>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       Gemm8Kvb::SMEM_BYTES) == cudaSuccess;
@@ -190,6 +204,11 @@ bool map_3d_bt(CUtensorMap* m, const void* base, uint64_t inner, uint64_t T, uin
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// How e4m3 weights meet bf16 activations (mla_set_e4m3_weight_conversion):
+// 0 = dequantised into a bf16 workspace copy per call, 1 = converted on chip
+// by the projection GEMMs.
+int g_e4m3_onchip = 0;
 
 // ------------------------------------------------------------------ profiling
 
@@ -376,8 +395,16 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
       w.attn8_s = take(rows * H * 4);
     }
   } else {
-    if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
-    if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+    if (!g_e4m3_onchip) {
+      if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
+      if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
+    } else {
+      // On-chip conversion: only the absorbed rows' GEMMs and decode read a
+      // bf16 copy of W_kvb (and decode one of W_o).
+      const int ng = (static_cast<int>(nq) + 3) / 4;
+      if (fp8 && ((attend && w.g_abs < ng) || dec)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
+      if (fp8 && dec) w.wo = take(H * kDv * kD * 2);
+    }
   }
   w.total = off;
   return w;
@@ -451,6 +478,57 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
   if (M <= Gemm2WoNarrow::BM)
     return launch_gemm_pair<Gemm2WoNarrow>(ds->pairs_wo_narrow, ta, tb, tc, M, N, K, ds->err, 4, st);
   return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st);
+}
+
+template <class Cfg>
+int launch_gemm_w8t(int pairs_max, const CUtensorMap& tx, const CUtensorMap& tw, const mla::GemmW8tArgs& g, int cls,
+                    cudaStream_t st) {
+  const int64_t ut = static_cast<int64_t>(Cfg::NT) * Cfg::BN;  // tokens per unit
+  const int64_t units = static_cast<int64_t>(g.F / Cfg::BM) * ((g.R + ut - 1) / ut);
+  const int pairs = units < pairs_max ? static_cast<int>(units) : pairs_max;
+  if (pairs <= 0) return MLA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+  const int rc = timed_launch(cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_w8t_kernel<Cfg>, tx, tw, g); });
+  return le != cudaSuccess ? MLA_ERR_CUDA : rc;
+}
+
+// kvh = latent . W_kvb^T with W_kvb as e4m3 codes [H*256, 512] and 128 x 128
+// block scales, converted on chip (no dequantised copy).
+int launch_gemm_w8t_kvb(const DeviceState* ds, int M, int H, const void* lat, const void* wkvb, const float* wkvb_s,
+                        void* kvh, bool v_f16, cudaStream_t st) {
+  const int N = H * (kDn + kDv), K = kL;
+  CUtensorMap tx, tw;
+  if (!map_2d(&tx, lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, GemmW8tKvb::HN) ||
+      !map_2d(&tw, wkvb, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    return MLA_ERR_CUDA;
+  const mla::GemmW8tArgs g = {wkvb_s, kvh, M, N, K, ds->err};
+  if (v_f16) return launch_gemm_w8t<GemmW8tKvbAttn>(ds->pairs_w8t_kvb, tx, tw, g, 2, st);
+  return launch_gemm_w8t<GemmW8tKvb>(ds->pairs_w8t_kvb, tx, tw, g, 2, st);
+}
+
+// out = attn . W_o with W_o as e4m3 codes [H*128, 7168] and block scales,
+// converted on chip.
+int launch_gemm_w8t_wo(const DeviceState* ds, int M, int H, const void* attn, const void* wo, const float* wo_s,
+                       void* out, cudaStream_t st) {
+  const int N = kD, K = H * kDv;
+  CUtensorMap tx, tw;
+  if (!map_2d(&tx, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, GemmW8tWo::HN) ||
+      !map_2d(&tw, wo, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, 128, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MLA_ERR_CUDA;
+  const mla::GemmW8tArgs g = {wo_s, out, M, N, K, ds->err};
+  return launch_gemm_w8t<GemmW8tWo>(ds->pairs_w8t_wo, tx, tw, g, 4, st);
 }
 
 // Dynamic e4m3 quantization of a bf16 [rows, cols] matrix: codes [rows, cols],
@@ -777,6 +855,7 @@ int run_upproject(const DeviceState* ds, const mla_dims& d, const WsLayout& lay,
   }
   const void* wk = W_kvb;
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    if (g_e4m3_onchip) return launch_gemm_w8t_kvb(ds, d.B * d.T, d.H, lat, W_kvb, W_kvb_scale, kvh, v_f16, st);
     void* dq = ws_at(ws, lay.wkvb);
     int rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st);
     if (rc != MLA_OK) return rc;
@@ -794,7 +873,11 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   const void* wk = W_kvb;
   int rc = MLA_OK;
   const bool act8 = d.act == MLA_ACT_E4M3_DYNAMIC;  // every row block-dense (absorbed_first_group)
-  if (d.wdtype == MLA_W_E4M3_BLOCK128 && !act8) {
+  // e4m3 W_kvb with bf16 activations: dequantised once into the workspace for
+  // every GEMM of the call, or, with on-chip conversion, only for the
+  // absorbed rows' absorb / un-absorb GEMMs (which read it as bf16).
+  const bool onchip = d.wdtype == MLA_W_E4M3_BLOCK128 && !act8 && g_e4m3_onchip;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128 && !act8 && (!onchip || lay.g_abs < ng)) {
     void* dq = ws_at(ws, lay.wkvb);
     rc = launch_dequant(ds, W_kvb, W_kvb_scale, dq, d.H * (kDn + kDv), kL, st);
     if (rc != MLA_OK) return rc;
@@ -803,8 +886,8 @@ int run_attend(const DeviceState* ds, const mla_dims& d, const WsLayout& lay, vo
   void* kvh = nullptr;
   if (lay.g_abs > 0) {  // up-projected keys, for the block-dense rows only
     kvh = ws_at(ws, lay.kvh);
-    rc = act8 ? run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, /*v_f16=*/true, st)
-              : launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, /*v_f16=*/true, st);
+    rc = (act8 || onchip) ? run_upproject(ds, d, lay, ws, lat, W_kvb, W_kvb_scale, kvh, /*v_f16=*/true, st)
+                          : launch_gemm_kvb(ds, d.B * d.T, d.H, lat, wk, kvh, /*v_f16=*/true, st);
     if (rc != MLA_OK) return rc;
   }
   void* bitmap = nullptr;
@@ -854,6 +937,8 @@ int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& la
     return launch_gemm8_wo(ds, M, d.H, attn8, attn_s, W_o, W_o_scale, out, st);
   }
   const void* wo = W_o;
+  if (d.wdtype == MLA_W_E4M3_BLOCK128 && g_e4m3_onchip)
+    return launch_gemm_w8t_wo(ds, d.B * d.T, d.H, attn, W_o, W_o_scale, out, st);
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
     void* dq = ws_at(ws, lay.wo);
     int rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st);
@@ -1060,6 +1145,12 @@ int mla_device_status(mla_stream_t stream, int* device_error) {
   if (cudaMemcpy(&v, ds->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
   if (v != 0 && cudaMemset(ds->err, 0, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
   *device_error = v;
+  return MLA_OK;
+}
+
+int mla_set_e4m3_weight_conversion(int onchip) {
+  if (onchip != 0 && onchip != 1) return MLA_ERR_SHAPE;
+  g_e4m3_onchip = onchip;
   return MLA_OK;
 }
 

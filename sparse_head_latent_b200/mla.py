@@ -58,6 +58,7 @@ SIGNATURES = {
     "mla_quantize_act": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP]),
     "mla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int)]),
+    "mla_set_e4m3_weight_conversion": (ctypes.c_int, [ctypes.c_int]),
     "mla_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
     "mla_test_withhold_attention_loads": (ctypes.c_int, [ctypes.c_int]),
     "mla_profile_begin": (ctypes.c_int, []),
@@ -267,6 +268,14 @@ def mla_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     _check("mla_device_status", load_library().mla_device_status(_stream(stream), ctypes.byref(v)))
     return v.value
+
+
+def mla_set_e4m3_weight_conversion(onchip: bool):
+    """e4m3 weights with bf16 activations: False (default) dequantises them
+    into a bf16 workspace copy per call; True converts them on chip inside
+    the projection GEMMs (bit-identical, no copy). Query workspace sizes
+    after switching."""
+    _check("mla_set_e4m3_weight_conversion", load_library().mla_set_e4m3_weight_conversion(1 if onchip else 0))
 
 
 def mla_set_wait_timeout_ns(ns: int):

@@ -66,6 +66,28 @@ def test_workspace_sizes(lib):
     assert mla.mla_workspace_bytes(d, 9, False) == 0
 
 
+def test_workspace_sizes_e4m3_weights_converted_on_chip(lib):
+    # With on-chip conversion the prefill GEMMs read the e4m3 codes directly:
+    # no dequantised copy for the up-projection, the output projection or a
+    # block-dense attend; the absorbed rows still get a bf16 copy of W_kvb.
+    d8 = _dims(wdtype=1, path=mla.MLA_PATH_BLOCK_DENSE)
+    dense_bf16 = mla.mla_workspace_bytes(_dims(path=mla.MLA_PATH_BLOCK_DENSE), mla.MLA_ENTRY_PREFILL, True)
+    absorbed = _dims(wdtype=1, path=mla.MLA_PATH_ABSORBED)
+    copy_kvb = 4 * 256 * 512 * 2
+    assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_PREFILL, True) == dense_bf16 + copy_kvb + 4 * 128 * 7168 * 2
+    mla.mla_set_e4m3_weight_conversion(True)
+    try:
+        assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_KV_UPPROJECT, False) == 0
+        assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_OUT_PROJECT, False) == 0
+        assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_PREFILL, True) == dense_bf16
+        abs_bf16 = mla.mla_workspace_bytes(_dims(path=mla.MLA_PATH_ABSORBED), mla.MLA_ENTRY_ATTEND, True)
+        assert mla.mla_workspace_bytes(absorbed, mla.MLA_ENTRY_ATTEND, True) == abs_bf16 + copy_kvb
+        assert lib.mla_set_e4m3_weight_conversion(2) == 2  # MLA_ERR_SHAPE
+    finally:
+        mla.mla_set_e4m3_weight_conversion(False)
+    assert mla.mla_workspace_bytes(d8, mla.MLA_ENTRY_KV_UPPROJECT, False) == copy_kvb
+
+
 def test_workspace_sizes_absorbed_path(lib):
     # Absorbed rows need no up-projected keys but q_abs and o_lat (rows x H x
     # 512 bf16 each) and the per-row key lists (k rounded up to 64, int32).

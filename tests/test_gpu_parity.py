@@ -104,23 +104,82 @@ def _dequant_bf16(codes, scale):
     return (f * scale[:, None, :, None]).view(R, C).to(torch.bfloat16)
 
 
+class _OnChip:
+    """Context: e4m3 weights with bf16 activations converted on chip by the
+    projection GEMMs (mla_set_e4m3_weight_conversion), restored on exit."""
+
+    def __init__(self, on):
+        self.on = on
+
+    def __enter__(self):
+        mla.mla_set_e4m3_weight_conversion(self.on)
+
+    def __exit__(self, *exc):
+        mla.mla_set_e4m3_weight_conversion(False)
+
+
+@pytest.mark.parametrize("onchip", [False, True], ids=["dequant", "onchip"])
 @pytest.mark.parametrize("stage", ["kv_upproject", "out_project"])
-def test_fp8_weight_gemms_equal_the_bf16_gemm_on_the_dequantised_weight(stage):
-    # With bf16 activations the e4m3 weight tiles are converted on chip
-    # (code exactly, times its 128 x 128 block scale in fp32, rounded to
-    # bf16) and fed to the bf16 tensor-core GEMM; the bf16 GEMM on the weight
-    # dequantised the same way on the host must give the same bits. Several
-    # row tiles (ragged), column tiles and 128-deep K blocks.
+def test_fp8_weight_gemms_equal_the_bf16_gemm_on_the_dequantised_weight(stage, onchip):
+    # With bf16 activations each e4m3 weight becomes bf16(code * block scale),
+    # the fp32 product rounded once, either in a dequantised copy or (onchip)
+    # by converter warps writing the tensor-core operand; the bf16 GEMM on
+    # the weight dequantised the same way on the host must give the same
+    # bits. Several row tiles (ragged), column tiles and 128-deep K blocks.
     x = synth.make_inputs(0, B=1, T=600, H=4, topk=None, seed=36, fp8=True)
     g = _dev(x)
     if stage == "kv_upproject":
-        got = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"], g["W_kvb_scale"])
+        with _OnChip(onchip):
+            got = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"], g["W_kvb_scale"])
         ref = mla.mla_kv_upproject(g["kv_latent"], _dequant_bf16(x.W_kvb, x.W_kvb_scale).cuda())
     else:
         gen = torch.Generator().manual_seed(37)
         attn = (0.05 * torch.randn(x.T, x.H * 128, generator=gen)).to(torch.bfloat16).cuda()
-        got = mla.mla_out_project(attn, g["W_o"], g["W_o_scale"])
+        with _OnChip(onchip):
+            got = mla.mla_out_project(attn, g["W_o"], g["W_o_scale"])
         ref = mla.mla_out_project(attn, _dequant_bf16(x.W_o, x.W_o_scale).cuda())
+    _no_device_error()
+    assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("stage", ["kv_upproject", "out_project"])
+def test_fp8_weight_gemms_bit_exact_over_many_units(stage):
+    # On-chip conversion with enough rows and heads that every CTA pair walks
+    # several work units: up-projection pairs cross from one 256-feature tile
+    # to the next inside their range (the weights converted into tensor
+    # memory are replaced), output-projection pairs take several 384-token
+    # units, and the last unit is ragged (4100 rows).
+    x = synth.make_inputs(0, B=1, T=4100, H=16, topk=None, seed=38, fp8=True)
+    g = _dev(x)
+    if stage == "kv_upproject":
+        with _OnChip(True):
+            got = mla.mla_kv_upproject(g["kv_latent"], g["W_kvb"], g["W_kvb_scale"])
+        ref = mla.mla_kv_upproject(g["kv_latent"], _dequant_bf16(x.W_kvb, x.W_kvb_scale).cuda())
+    else:
+        gen = torch.Generator().manual_seed(39)
+        attn = (0.05 * torch.randn(x.T, x.H * 128, generator=gen)).to(torch.bfloat16).cuda()
+        with _OnChip(True):
+            got = mla.mla_out_project(attn, g["W_o"], g["W_o_scale"])
+        ref = mla.mla_out_project(attn, _dequant_bf16(x.W_o, x.W_o_scale).cuda())
+    _no_device_error()
+    assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("path", [mla.MLA_PATH_BLOCK_DENSE, mla.MLA_PATH_AUTO], ids=["dense", "auto"])
+def test_prefill_with_e4m3_weights_converted_on_chip_equals_dequantised(path):
+    # The whole block with e4m3 weights: converting on chip must reproduce the
+    # dequantise-then-bf16 result bit for bit, also when some rows take the
+    # absorbed path (which keeps a bf16 copy of W_kvb for its GEMMs).
+    x = synth.make_inputs(0, B=2, T=1100, H=8, topk=48, seed=40, fp8=True)
+    g = _dev(x)
+
+    def run():
+        return mla.mla_prefill(g["q"], g["kv_latent"], g["k_pe"], g["W_kvb"], g["W_o"], g["W_kvb_scale"],
+                               g["W_o_scale"], topk_idx=g["topk_idx"], scale=x.scale, path=path)
+
+    ref = run()
+    with _OnChip(True):
+        got = run()
     _no_device_error()
     assert torch.equal(got, ref)
 
