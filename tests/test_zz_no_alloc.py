@@ -72,6 +72,32 @@ def test_static_scratch_entry_matches_workspace_entry_on_two_calls_in_a_row():
         assert torch.equal(got, ref), (x.T, path, act)
 
 
+@pytest.mark.gpu
+def test_static_scratch_entry_matches_the_oracle():
+    # The static entry against the fp64 oracle itself (every row, every
+    # head) for a block-dense and an absorbed problem, bf16 and e4m3
+    # weights, the e4m3 weights also with on-chip conversion (whose scratch
+    # holds no dequantised copy).
+    import oracle
+    lib = mla.load_library()
+    A, D = mla.MLA_PATH_ABSORBED, mla.MLA_PATH_BLOCK_DENSE
+    cases = [(synth.make_inputs(0, B=1, T=260, H=4, topk=40, seed=76), D, False),
+             (synth.make_inputs(0, B=1, T=700, H=4, topk=40, seed=77), A, False),
+             (synth.make_inputs(0, B=1, T=260, H=4, topk=40, seed=78, fp8=True), D, False),
+             (synth.make_inputs(0, B=1, T=260, H=4, topk=40, seed=78, fp8=True), D, True)]
+    for x, path, onchip in cases:
+        g = {k: v.cuda() for k, v in x.tensors().items()}
+        mla.mla_set_e4m3_weight_conversion(onchip)
+        try:
+            rc, got = _static_via_abi(lib, x, g, path)
+        finally:
+            mla.mla_set_e4m3_weight_conversion(False)
+        assert rc == 0, mla.mla_status_str(rc)
+        assert mla.mla_device_status() == 0
+        ref = oracle.attend_rows(x, list(range(x.B * x.T)))
+        _close(got.view(ref.shape), torch.from_numpy(ref))
+
+
 def test_static_scratch_entry_rejects_problems_beyond_its_scratch():
     # A host-side check that runs before any device work (no GPU needed).
     cuda_build.build()
