@@ -19,7 +19,7 @@
 // The pair computes D = W_tile . X_tile^T with one M = 256 UMMA per K step:
 // CTA r holds output features [128r, 128r+128) of the 256-feature tile as
 // tensor-memory lanes and the tokens [HN r, HN r + HN) of the token tile as
-// its half of the B operand (TMA, K-major, no multicast). Four converter
+// its half of the B operand (TMA, K-major, no multicast). Eight converter
 // warps per CTA read the e4m3 codes of their 128 features from shared
 // memory, scale, round to bf16 and store them into tensor memory (A operand,
 // lane = feature, column c = k pair (2c, 2c+1)); they arrive on the leader's
@@ -27,8 +27,8 @@
 // crosses between the two CTAs. Eight epilogue warps read D (lane = feature,
 // column = token); lane pairs trade values so that each lane holds two
 // adjacent features of one token, and the warp writes [token][feature] rows
-// with plain 32-bit stores (two 64-byte row segments per instruction: with
-// small TMA store boxes the per-store cost, not bandwidth, set the pace).
+// with plain 32-bit stores (two 64-byte row segments per instruction), so no
+// staging buffer is needed.
 //
 // Two forms:
 //   STATIONARY (K <= 512: the up-projection): a pair walks a contiguous range
@@ -55,8 +55,6 @@
 //   warps 10..17 epilogue: lanes 32 (w % 4) .. +31, alternate 32-token
 //               chunks ((w - 10) / 4)
 #pragma once
-
-#include <cuda_fp8.h>
 
 #include "gemm2.cuh"
 #include "ptx.cuh"
