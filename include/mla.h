@@ -168,7 +168,13 @@ int mla_attend(const mla_dims* dims, const void* q, const void* kv_latent,
  *   W_o  : bf16 or e4m3 [H*128, 7168] (math orientation [in, out]; a
  *          checkpoint's [out, in] weight is transposed once at load)
  *   W_o_scale: fp32 [H, 56] block scales for e4m3, else ignored
- *   out  : bf16 [B*T, 7168] */
+ *   out  : bf16 [B*T, 7168]
+ * With bf16 weights, more than 256 rows and K = H*128 >= 4096, the tiles of
+ * a last wave that would leave CTA pairs idle are split along K: their fp32
+ * partial tiles go to the workspace and a second kernel adds them in a
+ * fixed order. The result is deterministic for a given device and row
+ * count, but the rows of those tiles may round differently from a call
+ * with another row count. e4m3 weights keep whole-K tiles. */
 int mla_out_project(const mla_dims* dims, const void* attn, const void* W_o,
                     const float* W_o_scale, void* out, void* workspace,
                     size_t ws_bytes, mla_stream_t stream);
@@ -313,8 +319,9 @@ int mla_test_withhold_attention_loads(int on);
  * Classes: 0 topk prepass, 1 weight dequant, 2 W_kvb GEMM, 3 attention
  * (block-dense), 4 W_o GEMM, 5 per-row key lists (prefill and decode),
  * 6 absorb and un-absorb GEMMs, 7 attention (absorbed), 8 activation
- * quantization. Arrays must hold MLA_PROFILE_CLASSES entries. */
-#define MLA_PROFILE_CLASSES 9
+ * quantization, 9 sums of the W_o GEMM's K-split last-wave tiles. Arrays
+ * must hold MLA_PROFILE_CLASSES entries. */
+#define MLA_PROFILE_CLASSES 10
 int mla_profile_begin(void);
 int mla_profile_end(float* ms_total, int* launches);
 

@@ -65,6 +65,22 @@ struct GemmBatch {
   int c_col0, c_col_step;
 };
 
+// K-split of the last, partial wave of tiles (one plain GEMM only). When the
+// tile count T is not a multiple of the pair count P, the R = T mod P tiles
+// of the last wave would run on R pairs while the others idle. Instead the
+// T - R tiles of the whole waves run as usual and each of the R last tiles is
+// cut into `split` contiguous K ranges: pair p < R * split takes tile
+// T - R + p / split, range p % split, and writes its fp32 partial tile to
+// slot p of `part` (SPLIT_SLOT_FLOATS floats per slot). gemm_split_sum_kernel
+// then adds each tile's partials in range order into C. tail == 0: no split.
+struct GemmSplit {
+  float* part;
+  int tail;   // R
+  int split;  // K ranges per tile (>= 2 when tail > 0)
+};
+constexpr int SPLIT_SLOT_FLOATS = 256 * 256;  // one 256 x 256 tile
+constexpr GemmSplit kNoSplit = {nullptr, 0, 0};
+
 // Spin for about `ns` nanoseconds (used only to let in-flight copies land on
 // the abort path, where this CTA cannot observe the leader's barrier).
 __device__ __forceinline__ void spin_ns(uint64_t ns) {
@@ -76,7 +92,8 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, const GemmBatch bt, int* err) {
+                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, const GemmBatch bt,
+                     const GemmSplit sk, int* err) {
   constexpr int BK = Cfg::BK, S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,13 +145,34 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   const int num_kb = K / BK;
   const int pair = static_cast<int>(blockIdx.x) >> 1;
   const int num_pairs = static_cast<int>(gridDim.x) >> 1;
+  // This pair's work items: its whole tiles of the full waves, then (with a
+  // K-split tail) one K range of a last-wave tile. Item i gives the tile and
+  // the K-block range [kb0, kb1); the result says whether it is a K range.
+  const int full_end = num_tiles - sk.tail;
+  const int n_whole = pair < full_end ? (full_end - 1 - pair) / num_pairs + 1 : 0;
+  const int n_items = n_whole + (pair < sk.tail * sk.split ? 1 : 0);
+  auto item = [&](int i, int& tile, int& kb0, int& kb1) {
+    if (i < n_whole) {
+      tile = pair + i * num_pairs;
+      kb0 = 0;
+      kb1 = num_kb;
+      return false;
+    }
+    const int r = pair % sk.split;
+    tile = full_end + pair / sk.split;
+    kb0 = r * num_kb / sk.split;
+    kb1 = (r + 1) * num_kb / sk.split;
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (this CTA's halves)
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      for (int i = 0; i < n_items && ok; ++i) {
+        int tile, kb0, kb1;
+        item(i, tile, kb0, kb1);
         const int bi = tile / (num_m * num_n);
         int mt, nt;
         grouped_tile(tile - bi * num_m * num_n, num_m, num_n, Cfg::GROUP_M, mt, nt);
@@ -142,7 +180,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int bcol = nt * Cfg::BN + static_cast<int>(rank) * Cfg::HN;
         const int acol0 = bt.a_col0 + bi * bt.a_col_step;
         const int brow0 = bt.b_row0 + bi * bt.b_row_step;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1, ab, kErrWaitConsumer)) {
@@ -171,7 +209,9 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, Cfg::BN, 0, Cfg::B_MN_MAJOR ? 1 : 0);
       int it = 0, t = 0;
       bool ok = true;
-      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++t) {
+      for (int i = 0; i < n_items && ok; ++i, ++t) {
+        int tile, kb0, kb1;
+        item(i, tile, kb0, kb1);
         const int a = t & 1;
         const uint32_t aph = (t >> 1) & 1;
         if (!mbar_wait(acce0 + 8 * a, aph ^ 1, ab, kErrWaitEpilogue)) {
@@ -180,7 +220,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
         tc_fence_after();
         const uint32_t d = tmem_base + a * 256;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
           if (!mbar_wait(full0 + 8 * s, ph, ab, kErrWaitTma)) {
@@ -195,7 +235,7 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const uint64_t adesc = smem_desc_sw128(sa + k * 32, 16, 1024);
             const uint64_t bdesc = Cfg::B_MN_MAJOR ? smem_desc_sw128(sb + k * 16 * 128, BK * 128, 1024)
                                                    : smem_desc_sw128(sb + k * 32, 16, 1024);
-            umma_ss_pair(d, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_ss_pair(d, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit_pair(empty0 + 8 * s, 0x3);
         }
@@ -213,7 +253,9 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* bufs = epi + (warp - 2) * 2 * Cfg::EPI_BUF;
     int t = 0, nbuf = 0;
     float vmax = 0.f;  // largest |value| stored as f16 (V_F16)
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++t) {
+    for (int i = 0; i < n_items; ++i, ++t) {
+      int tile, kb0, kb1;
+      const bool ranged = item(i, tile, kb0, kb1);
       const int bi = tile / (num_m * num_n);
       int mt, nt;
       grouped_tile(tile - bi * num_m * num_n, num_m, num_n, Cfg::GROUP_M, mt, nt);
@@ -223,6 +265,32 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * 256;
       const int row0 = mt * Cfg::BM + static_cast<int>(rank) * Cfg::HM + q * 32;
+      if constexpr (Cfg::BN == 256 && !Cfg::V_F16) {
+        if (ranged) {
+          // fp32 partial of this warp's 32 rows in slot `pair`, laid out as
+          // [64 column quads][32 rows][4] so that every store of the warp
+          // covers 512 contiguous bytes.
+          float* dst = sk.part + static_cast<size_t>(pair) * SPLIT_SLOT_FLOATS + (rank * 4 + q) * 8192;
+#pragma unroll 1
+          for (int c = 0; c < 4 && row0 < M; ++c) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32x2(tb + c * 64, tb + c * 64 + 32, r0, r1);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              *reinterpret_cast<float4*>(dst + ((c * 16 + j) * 32 + lane) * 4) =
+                  make_float4(__uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1]),
+                              __uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3]));
+              *reinterpret_cast<float4*>(dst + ((c * 16 + 8 + j) * 32 + lane) * 4) =
+                  make_float4(__uint_as_float(r1[4 * j]), __uint_as_float(r1[4 * j + 1]),
+                              __uint_as_float(r1[4 * j + 2]), __uint_as_float(r1[4 * j + 3]));
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(mapa_shared(acce0 + 8 * a, 0));
+          continue;
+        }
+      }
       // A warp whose 32 rows all lie past M has nothing to store. It must
       // then skip the staging too: the two staging buffers alternate per
       // issued store, and `wait_group.read 1` before a buffer is rewritten
@@ -280,6 +348,39 @@ gemm_bf16_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   cluster_sync();  // the leader's UMMAs read the peer's shared memory until here
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+}
+
+// Second half of the K-split tail (GemmSplit): one thread per 4 output
+// columns of one row of a last-wave tile adds the tile's `split` partials in
+// K-range order (the same order for every element and every run) and stores
+// the bf16 result; rows past M are skipped. Thread e of the launch reads
+// element e % 16384 of each of its tile's slots, so the loads of a warp are
+// 512 contiguous bytes. C is row-major bf16 with row pitch ldc; the tile
+// order is the GEMM's (grouped_tile with group_m row tiles).
+__global__ void __launch_bounds__(256)
+gemm_split_sum_kernel(const float* __restrict__ part, __nv_bfloat16* __restrict__ C, int M, int ldc, int num_m,
+                      int num_n, int group_m, int first_tile, int tail, int split) {
+  const int e = static_cast<int>(blockIdx.x) * 256 + static_cast<int>(threadIdx.x);
+  if (e >= tail * (SPLIT_SLOT_FLOATS / 4)) return;
+  const int t = e / (SPLIT_SLOT_FLOATS / 4);
+  const int w = e - t * (SPLIT_SLOT_FLOATS / 4);  // [rank][warp][column quad][row] of the epilogue
+  const int row = (w & 31) + 32 * ((w >> 11) & 3) + 128 * (w >> 13);
+  const int quad = (w >> 5) & 63;
+  int mt, nt;
+  grouped_tile(first_tile + t, num_m, num_n, group_m, mt, nt);
+  const int grow = mt * 256 + row;
+  if (grow >= M) return;
+  const float4* p = reinterpret_cast<const float4*>(part) + static_cast<size_t>(t) * split * (SPLIT_SLOT_FLOATS / 4) + w;
+  float4 acc = p[0];
+  for (int r = 1; r < split; ++r) {
+    const float4 v = p[static_cast<size_t>(r) * (SPLIT_SLOT_FLOATS / 4)];
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  *reinterpret_cast<uint2*>(C + static_cast<size_t>(grow) * ldc + nt * 256 + quad * 4) =
+      make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
 }  // namespace mla

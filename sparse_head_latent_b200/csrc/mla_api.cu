@@ -269,6 +269,7 @@ struct WsLayout {
   size_t attn8 = kNone, attn8_s = kNone;  // e4m3 activations: quantized attention rows and scales
   int parts = 1;                          // decode: CTAs per (sequence, 64-head group)
   size_t wo_part = kNone;                 // decode: stream-K partial tiles of the output projection
+  size_t wo_split = kNone;                // prefill: partial tiles of the output projection's K-split last wave
   int g_abs = 0;       // first tile group on the absorbed path (groups of 4 x 128 query rows)
   int abs_chunk = 0;   // absorbed rows processed per pass
   int kpad = 0;        // pitch of the per-row key lists
@@ -283,6 +284,15 @@ constexpr int kAbsChunkRows = 2048;
 // on the device; a different count only changes how full the waves are).
 constexpr int kSmsForSplit = 148;
 constexpr int kStreamKCtas = 256;  // upper bound on the stream-K grid (the SM count)
+// K-split last wave of the prefill output projection (wo_split_plan): only
+// for K of at least kSplitMinTileKb 64-deep blocks (H >= 32; a shorter tile's
+// last wave ends before the partial sums would pay), each K range keeps at
+// least kSplitMinKb blocks, and the workspace holds kSplitSlots partial tiles
+// (the pair count of a 148-SM part; with more pairs the split only gets
+// coarser).
+constexpr int kSplitMinTileKb = 64;
+constexpr int kSplitMinKb = 8;
+constexpr int kSplitSlots = 74;
 // Cost model for MLA_PATH_AUTO: a tile group goes absorbed when its middle
 // row's causal prefix exceeds this many times the selection size. Measured
 // on B200 at T = 32768, H = 128, top-k 2048: the block-dense kernel costs
@@ -395,6 +405,11 @@ WsLayout ws_layout(const mla_dims& d, int entry, bool has_topk) {
       w.attn8_s = take(rows * H * 4);
     }
   } else {
+    // bf16 W_o over more than one row tile with a long K: partial tiles of
+    // the K-split last wave.
+    if (!fp8 && (entry == MLA_ENTRY_PREFILL || entry == MLA_ENTRY_OUT_PROJECT) && rows > 256 &&
+        static_cast<int>(H * kDv / 64) >= kSplitMinTileKb)
+      w.wo_split = take(static_cast<size_t>(kSplitSlots) * mla::SPLIT_SLOT_FLOATS * 4);
     if (!g_e4m3_onchip) {
       if (fp8 && (attend || dec || entry == MLA_ENTRY_KV_UPPROJECT)) w.wkvb = take(H * (kDn + kDv) * kL * 2);
       if (fp8 && (entry == MLA_ENTRY_PREFILL || dec || entry == MLA_ENTRY_OUT_PROJECT)) w.wo = take(H * kDv * kD * 2);
@@ -431,7 +446,8 @@ constexpr mla::GemmBatch kOneGemm = {1, 0, 0, 0, 0, 0, 0};
 
 template <class Cfg>
 int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M,
-                     int N, int K, int* err, int cls, cudaStream_t st, const mla::GemmBatch& bt = kOneGemm) {
+                     int N, int K, int* err, int cls, cudaStream_t st, const mla::GemmBatch& bt = kOneGemm,
+                     const mla::GemmSplit& sk = mla::kNoSplit) {
   const int tiles = ((M + Cfg::BM - 1) / Cfg::BM) * (N / Cfg::BN) * bt.count;
   const int pairs = tiles < pairs_max ? tiles : pairs_max;
   cudaLaunchConfig_t cfg = {};
@@ -448,7 +464,7 @@ int launch_gemm_pair(int pairs_max, const CUtensorMap& ta, const CUtensorMap& tb
   cfg.numAttrs = 1;
   cudaError_t le = cudaSuccess;
   const int rc = timed_launch(
-      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, bt, err); });
+      cls, st, [&] { le = cudaLaunchKernelEx(&cfg, mla::gemm_bf16_tc2_kernel<Cfg>, ta, tb, tc, M, N, K, bt, sk, err); });
   return le != cudaSuccess ? MLA_ERR_CUDA : rc;
 }
 
@@ -465,8 +481,32 @@ int launch_gemm_kvb(const DeviceState* ds, int M, int H, const void* lat, const 
   return launch_gemm_pair<Gemm2Kvb>(ds->pairs_kvb, ta, tb, tc, M, N, K, ds->err, 2, st);
 }
 
+// K-split of the output projection's last wave (mla::GemmSplit): how many
+// last-wave tiles are split (tail) and into how many K ranges (split), for a
+// grid of `pairs` CTA pairs. Each range keeps at least kSplitMinKb 64-deep K
+// blocks, and tail * split stays within the kSplitSlots partial tiles the
+// workspace holds; no split (tail 0) when K is short, the waves are whole or
+// fewer than two ranges would result.
+mla::GemmSplit wo_split_plan(int tiles, int pairs, int num_kb, float* part) {
+  mla::GemmSplit sk = mla::kNoSplit;
+  if (part == nullptr || pairs <= 0 || num_kb < kSplitMinTileKb) return sk;
+  const int tail = tiles % pairs;
+  if (tail == 0) return sk;
+  int split = pairs / tail;
+  if (split > num_kb / kSplitMinKb) split = num_kb / kSplitMinKb;
+  if (split > kSplitSlots / tail) split = kSplitSlots / tail;
+  if (split < 2) return sk;
+  sk.part = part;
+  sk.tail = tail;
+  sk.split = split;
+  return sk;
+}
+
+// split_part: kSplitSlots * SPLIT_SLOT_FLOATS fp32 of workspace for the
+// K-split last wave, or nullptr (every tile whole, e.g. so that the result
+// matches another kernel's whole-K tiles bit for bit).
 int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const void* wo, void* out,
-                   cudaStream_t st) {
+                   cudaStream_t st, float* split_part = nullptr) {
   const int N = kD, K = H * kDv;
   CUtensorMap ta, tb, tc;
   if (!map_2d(&ta, attn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(K) * 2, 64, 128) ||
@@ -477,7 +517,18 @@ int launch_gemm_wo(const DeviceState* ds, int M, int H, const void* attn, const 
   // idle while W_o streams through; 128-wide tiles double the pairs.
   if (M <= Gemm2WoNarrow::BM)
     return launch_gemm_pair<Gemm2WoNarrow>(ds->pairs_wo_narrow, ta, tb, tc, M, N, K, ds->err, 4, st);
-  return launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st);
+  const int num_m = (M + Gemm2Wo::BM - 1) / Gemm2Wo::BM, num_n = N / Gemm2Wo::BN;
+  const int tiles = num_m * num_n;
+  const int pairs = tiles < ds->pairs_wo ? tiles : ds->pairs_wo;
+  const mla::GemmSplit sk = wo_split_plan(tiles, pairs, K / Gemm2Wo::BK, split_part);
+  int rc = launch_gemm_pair<Gemm2Wo>(ds->pairs_wo, ta, tb, tc, M, N, K, ds->err, 4, st, kOneGemm, sk);
+  if (rc != MLA_OK || sk.tail == 0) return rc;
+  const int threads = sk.tail * (mla::SPLIT_SLOT_FLOATS / 4);
+  return timed_launch(9, st, [&] {
+    mla::gemm_split_sum_kernel<<<(threads + 255) / 256, 256, 0, st>>>(
+        sk.part, static_cast<__nv_bfloat16*>(out), M, N, num_m, num_n, Gemm2Wo::GROUP_M, tiles - sk.tail, sk.tail,
+        sk.split);
+  });
 }
 
 template <class Cfg>
@@ -940,12 +991,14 @@ int run_out_project(const DeviceState* ds, const mla_dims& d, const WsLayout& la
   if (d.wdtype == MLA_W_E4M3_BLOCK128 && g_e4m3_onchip)
     return launch_gemm_w8t_wo(ds, d.B * d.T, d.H, attn, W_o, W_o_scale, out, st);
   if (d.wdtype == MLA_W_E4M3_BLOCK128) {
+    // Whole-K tiles only, so that both e4m3 conversion modes give the same bits.
     void* dq = ws_at(ws, lay.wo);
     int rc = launch_dequant(ds, W_o, W_o_scale, dq, d.H * kDv, kD, st);
     if (rc != MLA_OK) return rc;
-    wo = dq;
+    return launch_gemm_wo(ds, d.B * d.T, d.H, attn, dq, out, st);
   }
-  return launch_gemm_wo(ds, d.B * d.T, d.H, attn, wo, out, st);
+  float* split = lay.wo_split == kNone ? nullptr : reinterpret_cast<float*>(ws_at(ws, lay.wo_split));
+  return launch_gemm_wo(ds, d.B * d.T, d.H, attn, wo, out, st, split);
 }
 
 // Decode: one new query per sequence (row s = T-1) against the cache, in the

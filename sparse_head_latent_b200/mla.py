@@ -20,11 +20,11 @@ _lib = None
 
 MLA_ENTRY_KV_UPPROJECT, MLA_ENTRY_ATTEND, MLA_ENTRY_OUT_PROJECT, MLA_ENTRY_PREFILL, MLA_ENTRY_DECODE = 0, 1, 2, 3, 4
 MLA_W_BF16, MLA_W_E4M3_BLOCK128 = 0, 1
-MLA_PROFILE_CLASSES = 9
+MLA_PROFILE_CLASSES = 10
 MLA_PATH_AUTO, MLA_PATH_BLOCK_DENSE, MLA_PATH_ABSORBED = 0, 1, 2
 MLA_ACT_BF16, MLA_ACT_E4M3_DYNAMIC = 0, 1
 PROFILE_CLASS_NAMES = ("topk_prepass", "weight_dequant", "gemm_kvb", "attention", "gemm_wo", "row_lists",
-                       "gemm_absorb", "attention_absorbed", "act_quant")
+                       "gemm_absorb", "attention_absorbed", "act_quant", "gemm_wo_split_sum")
 D_NOPE, D_ROPE, D_V, D_LATENT, D_MODEL = 128, 64, 128, 512, 7168
 
 

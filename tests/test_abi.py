@@ -66,6 +66,34 @@ def test_workspace_sizes(lib):
     assert mla.mla_workspace_bytes(d, 9, False) == 0
 
 
+def test_workspace_sizes_output_projection_split(lib):
+    # bf16 W_o with K >= 4096 (H >= 32) over more than one 256-row tile keeps
+    # 74 fp32 256 x 256 partial tiles for the K-split last wave; short K, a
+    # single row tile, e4m3 weights (whole-K tiles, the same bits in both
+    # conversion modes) and e4m3 activations (their own GEMM) keep none.
+    slots = 74 * 256 * 256 * 4
+
+    def ws(B, T, H, entry, topk=False, **kw):
+        d = mla.make_dims(B, T, H, 16 if topk else 0, False)
+        for k, v in kw.items():
+            setattr(d, k, v)
+        return mla.mla_workspace_bytes(d, entry, topk)
+
+    assert ws(1, 600, 32, mla.MLA_ENTRY_OUT_PROJECT) == slots
+    assert ws(2, 300, 128, mla.MLA_ENTRY_OUT_PROJECT) == slots
+    assert ws(1, 600, 16, mla.MLA_ENTRY_OUT_PROJECT) == 0
+    assert ws(1, 256, 128, mla.MLA_ENTRY_OUT_PROJECT) == 0
+    assert ws(1, 600, 32, mla.MLA_ENTRY_OUT_PROJECT, wdtype=1) == 32 * 128 * 7168 * 2
+    assert ws(1, 600, 32, mla.MLA_ENTRY_OUT_PROJECT, wdtype=1, act=mla.MLA_ACT_E4M3_DYNAMIC) == (
+        600 * 32 * 128 + 600 * 32 * 4)
+    dense = mla.MLA_PATH_BLOCK_DENSE
+    attend = ws(1, 600, 32, mla.MLA_ENTRY_ATTEND, True, path=dense)
+    attn_rows = 600 * 32 * 128 * 2
+    assert ws(1, 600, 32, mla.MLA_ENTRY_PREFILL, True, path=dense) == attend + attn_rows + slots
+    assert ws(1, 600, 32, mla.MLA_ENTRY_ATTEND, False, path=dense) == 600 * 32 * 256 * 2
+    assert ws(1, 600, 32, mla.MLA_ENTRY_KV_UPPROJECT) == 0
+
+
 def test_workspace_sizes_e4m3_weights_converted_on_chip(lib):
     # With on-chip conversion the prefill GEMMs read the e4m3 codes directly:
     # no dequantised copy for the up-projection, the output projection or a

@@ -97,6 +97,31 @@ def test_output_projection_matches_oracle(rows, H, fp8):
     assert_close(out.float().cpu().numpy(), ref, "out")
 
 
+@pytest.mark.parametrize("rows,H", [(600, 32), (1300, 128)])
+def test_output_projection_with_k_split_last_wave_matches_oracle(rows, H):
+    # bf16 W_o with K = H * 128 >= 4096 and a tile count that leaves the last
+    # wave of CTA pairs partial (600 rows: 84 tiles of 256 x 256, 10 of them
+    # in the last wave on 74 pairs; 1300 rows: 168 tiles, 20): those tiles are
+    # cut along K, and a second kernel adds their fp32 partials. Whole rows
+    # cover every column tile (whole and split ones), the ragged last row
+    # tile included; a repeat must give the same bits.
+    x = synth.make_inputs(0, T=8, H=H, topk=None, seed=23)
+    gen = torch.Generator().manual_seed(rows)
+    attn = (0.05 * torch.randn(rows, H * 128, generator=gen)).to(torch.bfloat16)
+    g = _dev(x)
+    mla.mla_profile_begin()
+    out = mla.mla_out_project(attn.cuda(), g["W_o"])
+    prof = mla.mla_profile_end()
+    _no_device_error()
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert prof["gemm_wo_split_sum"][1] == 1
+    sample = sorted({0, 1, 127, 128, 255, 256, 511, 512, rows // 2, rows - 2, rows - 1})
+    ref = oracle.project_rows(x, attn[sample].to(torch.float64).numpy())
+    assert_close(out[sample].float().cpu().numpy(), ref, "out")
+    assert torch.equal(mla.mla_out_project(attn.cuda(), g["W_o"]), out)
+    _no_device_error()
+
+
 def _dequant_bf16(codes, scale):
     """bf16(e4m3(code) * block scale), the fp32 product rounded to nearest even."""
     R, C = codes.shape
