@@ -311,6 +311,16 @@ int mla_set_wait_timeout_ns(unsigned long long ns);
  * like mla_set_wait_timeout_ns; switch it off again before normal use. */
 int mla_test_withhold_attention_loads(int on);
 
+/* Test hook, host only (no device work): the plan mla_out_project and
+ * mla_prefill use for a W_o GEMM of `tiles` 256 x 256 tiles on `pairs` CTA
+ * pairs with K of `num_kb` 64-deep blocks (bf16 weights, more than 256
+ * rows): *tail tiles of the last wave, each cut into *split contiguous K
+ * ranges, one per pair, the partial tiles in the first tail * split of the
+ * workspace's 74 slots; 0 and 0 for no split. tail and split are HOST
+ * pointers. Returns MLA_ERR_NULL if one is NULL, MLA_ERR_SHAPE if an
+ * argument is negative. */
+int mla_test_wo_split_plan(int tiles, int pairs, int num_kb, int* tail, int* split);
+
 /* Per-kernel device timing (CUDA events on the launching stream).
  * mla_profile_begin() starts recording events around every launch made by
  * the calls above on this host thread's library instance; mla_profile_end()

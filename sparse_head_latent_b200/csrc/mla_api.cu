@@ -1221,6 +1221,16 @@ int mla_test_withhold_attention_loads(int on) {
   return cudaMemcpyToSymbol(mla::g_mla_withhold_attn_loads, &v, sizeof v) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+int mla_test_wo_split_plan(int tiles, int pairs, int num_kb, int* tail, int* split) {
+  if (tail == nullptr || split == nullptr) return MLA_ERR_NULL;
+  if (tiles < 0 || pairs < 0 || num_kb < 0) return MLA_ERR_SHAPE;
+  float dummy = 0.f;  // any non-null workspace pointer: the plan only tests it for null
+  const mla::GemmSplit sk = wo_split_plan(tiles, pairs, num_kb, &dummy);
+  *tail = sk.tail;
+  *split = sk.split;
+  return MLA_OK;
+}
+
 int mla_profile_begin(void) {
   for (auto& r : t_prof.recs) {
     t_prof.pool.push_back(r.start);

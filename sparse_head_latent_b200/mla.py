@@ -61,6 +61,8 @@ SIGNATURES = {
     "mla_set_e4m3_weight_conversion": (ctypes.c_int, [ctypes.c_int]),
     "mla_set_wait_timeout_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
     "mla_test_withhold_attention_loads": (ctypes.c_int, [ctypes.c_int]),
+    "mla_test_wo_split_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "mla_profile_begin": (ctypes.c_int, []),
     "mla_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
 }

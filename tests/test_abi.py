@@ -278,3 +278,49 @@ def test_static_scratch_limit_agrees_with_the_library(lib):
     if torch.cuda.is_available():
         pytest.skip("the accepted case would launch kernels on placeholder pointers")
     assert call(fits) not in (0, 8)  # passes the size check, then finds no usable device
+
+
+def _split_plan(lib, tiles, pairs, num_kb):
+    tail, split = ctypes.c_int(-1), ctypes.c_int(-1)
+    assert lib.mla_test_wo_split_plan(tiles, pairs, num_kb, ctypes.byref(tail), ctypes.byref(split)) == 0
+    return tail.value, split.value
+
+
+def test_output_projection_split_plan_covers_every_k_block_once(lib):
+    # The library's own plan for the W_o GEMM's K-split last wave, walked the
+    # way the kernel assigns work (pair p: whole tiles p, p + P, ... below
+    # T - R, then range p % S of tile T - R + p / S for p < R * S, K blocks
+    # [r * kb / S, (r + 1) * kb / S)): every (tile, K block) exactly once,
+    # at most 74 partial slots, ranges of at least 8 blocks, and no split for
+    # K below 64 blocks or whole waves.
+    assert _split_plan(lib, 448, 74, 256) == (4, 18)      # T=4096, H=128 on 148 SMs
+    assert _split_plan(lib, 896, 74, 128) == (8, 9)       # T=8192, H=64
+    assert _split_plan(lib, 448, 74, 32) == (0, 0)        # K = 2048: too short to pay
+    assert _split_plan(lib, 444, 74, 256) == (0, 0)       # whole waves
+    assert _split_plan(lib, 120, 74, 256) == (0, 0)       # 46 tiles left: one range each
+    for tiles in (1, 2, 28, 56, 84, 140, 224, 448, 476, 896, 1792, 3584):
+        for pairs in (1, 3, 37, 60, 74, 100, 148):
+            for num_kb in (8, 63, 64, 100, 128, 256, 512):
+                P = min(tiles, pairs)
+                tail, split = _split_plan(lib, tiles, P, num_kb)
+                if tail == 0:
+                    assert split == 0
+                    continue
+                assert num_kb >= 64 and tail == tiles % P and 2 <= split <= P // tail
+                assert tail * split <= 74 and num_kb // split >= 8
+                seen = set()
+                full_end = tiles - tail
+                for p in range(P):
+                    for t in range(p, full_end, P):
+                        seen.update((t, kb) for kb in range(num_kb))
+                    if p < tail * split:
+                        r, t = p % split, full_end + p // split
+                        kb0, kb1 = r * num_kb // split, (r + 1) * num_kb // split
+                        assert kb1 > kb0
+                        before = len(seen)
+                        seen.update((t, kb) for kb in range(kb0, kb1))
+                        assert len(seen) == before + kb1 - kb0
+                assert len(seen) == tiles * num_kb
+    tail = ctypes.c_int()
+    assert lib.mla_test_wo_split_plan(448, 74, 256, ctypes.byref(tail), None) == 1
+    assert lib.mla_test_wo_split_plan(-1, 74, 256, ctypes.byref(tail), ctypes.byref(tail)) == 2
