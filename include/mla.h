@@ -3,7 +3,7 @@
  *
  * The block is the full-sequence (prefill) path of multi-head latent
  * attention as given on the DeepSeek-V3.2-Exp "Sparse attention" page
- * (model.py 574-589, 607-608) and the Kimi K2 "Output projection" page:
+ * (its prefill code) and the Kimi K2 "Output projection" page:
  *
  *   [k_nope_h | v_h][t] = W_kvb,h . kv_latent[t]              (wkv_b, view, split)
  *   k_h[t]              = k_nope_h[t] ++ k_pe[t]                (rotary key shared by heads)

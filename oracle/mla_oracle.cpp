@@ -6,8 +6,8 @@
 // CPU-baseline leg of the benchmark do. It shares no code, header or table
 // with the CUDA library.
 //
-// What it computes (DeepSeek-V3.2-Exp "Sparse attention" page, prefill code
-// of model.py 574-589 and 607-608; Kimi K2 "Output projection" page):
+// What it computes (DeepSeek-V3.2-Exp "Sparse attention" page, its prefill
+// code; Kimi K2 "Output projection" page):
 //   kv            = W_kvb applied to the 512-wide latent, viewed per head as
 //                   [k_nope (128) | v (128)]                     (wkv_b, view, split)
 //   k_h[t]        = k_nope_h[t] ++ k_pe[t]  (rotary key shared by all heads)
